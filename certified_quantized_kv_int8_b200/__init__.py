@@ -1,0 +1,324 @@
+"""Python binding of libcqa.so: certified quantized KV-cache decode attention on B200.
+
+Argument marshalling only.  Every step of the decode path runs in the CUDA
+library; torch is used for device buffers and streams.  The functions carry
+the names of the C entry points declared in include/cqa.h:
+
+    cqa_cache_create, cqa_cache_destroy, cqa_cache_length,
+    cqa_quantize_append, cqa_decode, cqa_dense_reference,
+    cqa_debug_export, cqa_error_string
+
+and ``Cache`` wraps a handle with the same calls as methods.  Importing this
+module does not load the library; the first call does, and fails loudly if
+libcqa.so has not been built (``python -m certified_quantized_kv_int8_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass, asdict
+
+import numpy as np
+import torch
+
+from .build import LIB
+
+__all__ = [
+    "CqaError", "Thresholds", "Cache", "load_library",
+    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
+    "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
+    "cqa_profile_begin", "cqa_profile_end", "PHASES",
+    "EXPORT_KCODES", "EXPORT_KSCALE", "EXPORT_VCODES", "EXPORT_VMETA", "EXPORT_ETA",
+    "EXPORT_VRANGE", "EXPORT_RESIDUAL", "EXPORT_TIER2",
+]
+
+EXPORT_KCODES, EXPORT_KSCALE, EXPORT_VCODES, EXPORT_VMETA = 0, 1, 2, 3
+EXPORT_ETA, EXPORT_VRANGE, EXPORT_RESIDUAL, EXPORT_TIER2 = 4, 5, 6, 7
+
+EXPORTED_SYMBOLS = (
+    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
+    "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
+    "cqa_profile_begin", "cqa_profile_end",
+)
+
+PHASES = ("append_seal", "append_tail", "score", "select", "attend", "combine",
+          "dense_attend", "dense_combine")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+                ("device", ctypes.c_int32)]
+
+
+class _Thresholds(ctypes.Structure):
+    _fields_ = [("tau_cov", ctypes.c_float), ("eps_key", ctypes.c_float),
+                ("max_expand", ctypes.c_int32), ("v_tol", ctypes.c_float),
+                ("rank_r", ctypes.c_int32), ("eps_val", ctypes.c_float),
+                ("layer_dense_frac", ctypes.c_float), ("naive", ctypes.c_int32)]
+
+
+class _Trace(ctypes.Structure):
+    _fields_ = [("kstar", ctypes.c_void_p), ("block_flags", ctypes.c_void_p),
+                ("ell8", ctypes.c_void_p), ("ell16", ctypes.c_void_p),
+                ("delta", ctypes.c_void_p), ("head_flags", ctypes.c_void_p),
+                ("ell_res", ctypes.c_void_p)]
+
+
+@dataclass
+class Thresholds:
+    """Decode thresholds (see cqa_thresholds in include/cqa.h)."""
+
+    tau_cov: float = 0.995
+    eps_key: float = 5e-3
+    max_expand: int = 4
+    v_tol: float = 0.05
+    rank_r: int = 4
+    eps_val: float = float("inf")
+    layer_dense_frac: float = 0.5
+    naive: bool = False
+
+    def as_c(self) -> _Thresholds:
+        return _Thresholds(self.tau_cov, self.eps_key, int(self.max_expand), self.v_tol,
+                           int(self.rank_r), self.eps_val, self.layer_dense_frac,
+                           1 if self.naive else 0)
+
+    def float32_rounded(self) -> dict:
+        """The values the library sees (floats rounded to float32), as a dict."""
+        d = asdict(self)
+        for k in ("tau_cov", "eps_key", "v_tol", "eps_val", "layer_dense_frac"):
+            d[k] = float(np.float32(d[k]))
+        return d
+
+
+class CqaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {cqa_error_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libcqa.so (built in-tree); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise RuntimeError(
+            f"{LIB} is missing: build it with `python -m certified_quantized_kv_int8_b200.build`")
+    lib = ctypes.CDLL(LIB)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    lib.cqa_cache_create.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(vp)]
+    lib.cqa_cache_destroy.argtypes = [vp]
+    lib.cqa_cache_length.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.cqa_quantize_append.argtypes = [vp, i32, vp, vp, i32, vp]
+    lib.cqa_decode.argtypes = [vp, i32, vp, ctypes.POINTER(_Thresholds), vp, vp, vp, vp,
+                               ctypes.POINTER(_Trace), vp]
+    lib.cqa_dense_reference.argtypes = [vp, i32, vp, vp, vp]
+    lib.cqa_debug_export.argtypes = [vp, i32, i32, vp, ctypes.c_size_t]
+    lib.cqa_debug_export.restype = ctypes.c_int64
+    lib.cqa_profile_begin.argtypes = [vp, i32]
+    lib.cqa_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_int64)]
+    lib.cqa_error_string.argtypes = [i32]
+    lib.cqa_error_string.restype = ctypes.c_char_p
+    for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
+                 "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
+                 "cqa_profile_begin", "cqa_profile_end"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(code: int, where: str):
+    if code < 0:
+        raise CqaError(code, where)
+    return code
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, shape, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name}: expected a contiguous {dtype} CUDA tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def cqa_error_string(code: int) -> str:
+    return load_library().cqa_error_string(int(code)).decode()
+
+
+def cqa_cache_create(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0):
+    cfg = _Config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device)
+    h = ctypes.c_void_p()
+    _check(load_library().cqa_cache_create(ctypes.byref(cfg), ctypes.byref(h)), "cqa_cache_create")
+    return h
+
+
+def cqa_cache_destroy(handle):
+    return _check(load_library().cqa_cache_destroy(handle), "cqa_cache_destroy")
+
+
+def cqa_cache_length(handle, layer: int) -> int:
+    out = ctypes.c_int32()
+    _check(load_library().cqa_cache_length(handle, layer, ctypes.byref(out)), "cqa_cache_length")
+    return int(out.value)
+
+
+def cqa_quantize_append(handle, layer, k, v, stream=None):
+    """k, v: CUDA float16 [batch][n_kv_heads][n_new][head_dim]."""
+    n_new = int(k.shape[2])
+    return _check(load_library().cqa_quantize_append(handle, layer, _ptr(k), _ptr(v), n_new,
+                                                     _stream(stream)), "cqa_quantize_append")
+
+
+def cqa_decode(handle, layer, q, th: Thresholds, out, e_key, e_val, rung, trace=None, stream=None):
+    """q: CUDA float16 [batch][n_q_heads][head_dim]; out float32 like q; e_key, e_val float32
+    [batch][n_q_heads]; rung uint8 [batch][n_q_heads].  trace: dict of CUDA tensors keyed by
+    the cqa_trace field names (any subset)."""
+    tr = None
+    if trace:
+        tr = _Trace(**{k: (v.data_ptr() if v is not None else None) for k, v in trace.items()})
+    return _check(load_library().cqa_decode(
+        handle, layer, _ptr(q), ctypes.byref(th.as_c()), _ptr(out), _ptr(e_key), _ptr(e_val),
+        _ptr(rung), ctypes.byref(tr) if tr is not None else None, _stream(stream)), "cqa_decode")
+
+
+def cqa_dense_reference(handle, layer, q, out, stream=None):
+    return _check(load_library().cqa_dense_reference(handle, layer, _ptr(q), _ptr(out),
+                                                     _stream(stream)), "cqa_dense_reference")
+
+
+def cqa_debug_export(handle, layer, what, dst: np.ndarray | None = None):
+    """Copy one Tier-1 array to a numpy buffer (synchronous); with dst None return its size."""
+    lib = load_library()
+    if dst is None:
+        return _check(lib.cqa_debug_export(handle, layer, what, None, 0), "cqa_debug_export")
+    return _check(lib.cqa_debug_export(handle, layer, what, dst.ctypes.data_as(ctypes.c_void_p),
+                                       dst.nbytes), "cqa_debug_export")
+
+
+def cqa_profile_begin(handle, max_launches: int = 1 << 16):
+    return _check(load_library().cqa_profile_begin(handle, int(max_launches)), "cqa_profile_begin")
+
+
+def cqa_profile_end(handle):
+    """Returns ({phase: ms}, {phase: launches}, untimed launches)."""
+    ms = (ctypes.c_double * len(PHASES))()
+    n = (ctypes.c_int64 * len(PHASES))()
+    untimed = _check(load_library().cqa_profile_end(handle, ms, n), "cqa_profile_end")
+    return ({p: ms[i] for i, p in enumerate(PHASES)}, {p: int(n[i]) for i, p in enumerate(PHASES)},
+            untimed)
+
+
+class Cache:
+    """A cqa_cache handle with its shape; methods mirror the C entry points."""
+
+    def __init__(self, n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0):
+        self.n_layers, self.batch = n_layers, batch
+        self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
+        self.max_ctx, self.device = max_ctx, device
+        self.handle = cqa_cache_create(n_layers, batch, n_q_heads, n_kv_heads, head_dim,
+                                       max_ctx, device)
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            cqa_cache_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def profile_begin(self, max_launches: int = 1 << 16):
+        return cqa_profile_begin(self.handle, max_launches)
+
+    def profile_end(self):
+        return cqa_profile_end(self.handle)
+
+    def length(self, layer):
+        return cqa_cache_length(self.handle, layer)
+
+    def append(self, layer, k, v, stream=None):
+        B, H, d = self.batch, self.n_kv_heads, self.head_dim
+        _dev(k, torch.float16, (B, H, k.shape[2], d), "k")
+        _dev(v, torch.float16, (B, H, k.shape[2], d), "v")
+        return cqa_quantize_append(self.handle, layer, k, v, stream)
+
+    def alloc_outputs(self):
+        dev = torch.device("cuda", self.device)
+        B, Hq, d = self.batch, self.n_q_heads, self.head_dim
+        return (torch.empty(B, Hq, d, dtype=torch.float32, device=dev),
+                torch.empty(B, Hq, dtype=torch.float32, device=dev),
+                torch.empty(B, Hq, dtype=torch.float32, device=dev),
+                torch.empty(B, Hq, dtype=torch.uint8, device=dev))
+
+    def alloc_trace(self, layer):
+        dev = torch.device("cuda", self.device)
+        B, Hq, Hkv = self.batch, self.n_q_heads, self.n_kv_heads
+        nb = max(1, self.length(layer) // 64)
+        return dict(
+            kstar=torch.empty(B, Hq, dtype=torch.int32, device=dev),
+            block_flags=torch.empty(B, Hkv, nb, dtype=torch.uint8, device=dev),
+            ell8=torch.empty(B, Hq, nb, dtype=torch.float32, device=dev),
+            ell16=torch.full((B, Hq, nb), math.nan, dtype=torch.float32, device=dev),
+            delta=torch.empty(B, Hq, nb, dtype=torch.float32, device=dev),
+            head_flags=torch.empty(B, Hq, dtype=torch.uint8, device=dev),
+            ell_res=torch.empty(B, Hq, dtype=torch.float32, device=dev),
+        )
+
+    def decode(self, layer, q, th: Thresholds, outputs=None, trace=None, stream=None):
+        B, Hq, d = self.batch, self.n_q_heads, self.head_dim
+        _dev(q, torch.float16, (B, Hq, d), "q")
+        out, e_key, e_val, rung = outputs if outputs is not None else self.alloc_outputs()
+        cqa_decode(self.handle, layer, q, th, out, e_key, e_val, rung, trace, stream)
+        return out, e_key, e_val, rung
+
+    def dense_reference(self, layer, q, out=None, stream=None):
+        B, Hq, d = self.batch, self.n_q_heads, self.head_dim
+        _dev(q, torch.float16, (B, Hq, d), "q")
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        cqa_dense_reference(self.handle, layer, q, out, stream)
+        return out
+
+    def export(self, layer, what):
+        """Tier-1 array of `layer` as a numpy array shaped per include/cqa.h."""
+        B, H, d = self.batch, self.n_kv_heads, self.head_dim
+        T = self.length(layer)
+        nb, r = T // 64, T % 64
+        spec = {
+            EXPORT_KCODES: (np.int8, (B, H, nb, 64, d)),
+            EXPORT_KSCALE: (np.float32, (B, H, nb, d)),
+            EXPORT_VCODES: (np.uint8, (B, H, nb, 64, d // 2)),
+            EXPORT_VMETA: (np.float32, (B, H, nb, 64, d // 32, 2)),
+            EXPORT_ETA: (np.float32, (B, H, nb)),
+            EXPORT_VRANGE: (np.float32, (B, H, 2, d)),
+            EXPORT_RESIDUAL: (np.float16, (B, H, 2, r, d)),
+            EXPORT_TIER2: (np.float16, (B, H, 2, T, d)),
+        }[what]
+        dst = np.empty(spec[1], dtype=spec[0])
+        n = cqa_debug_export(self.handle, layer, what, dst)
+        assert n == dst.nbytes
+        return dst

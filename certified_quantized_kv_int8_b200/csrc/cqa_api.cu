@@ -1,0 +1,498 @@
+// C ABI of libcqa.so: cache management, argument checks, launch sequences.
+// The declarations and their contracts are in include/cqa.h.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "cqa_internal.cuh"
+
+namespace cqa {
+size_t select_smem_bytes(int G, int nb);
+}
+
+using namespace cqa;
+
+struct cqa_cache {
+  cqa_config cfg;
+  int G, nbm;
+  Strides st;
+  Tier1 t;
+  Scratch sc;
+  int32_t* len;  // host: tokens per layer
+  void* k2_host;
+  void* v2_host;
+  size_t tier2_bytes;  // per tier-2 array
+  void* dev_block;     // one device allocation holding Tier 1 and scratch
+  // profiling (cqa_profile_begin / cqa_profile_end)
+  bool prof_on;
+  std::vector<cudaEvent_t>* prof_events;
+  std::vector<int>* prof_phase;
+  size_t prof_max;
+  int64_t prof_launches[CQA_PHASE_COUNT];
+  int64_t prof_untimed;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) ok = true;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+constexpr int kTargetCtas = 148 * 4;  // attend grid target: several waves over 148 SMs
+
+void chunking(int units, int nb, int* chunk_blocks, int* nchunks) {
+  int per_unit = (kTargetCtas + units - 1) / units;
+  if (per_unit < 1) per_unit = 1;
+  int cb = nb > 0 ? (nb + per_unit - 1) / per_unit : 1;
+  if (cb < 1) cb = 1;
+  *chunk_blocks = cb;
+  int nc = nb > 0 ? (nb + cb - 1) / cb : 1;
+  *nchunks = nc < 1 ? 1 : nc;
+}
+
+int max_chunks_for(int units) { return (kTargetCtas + units - 1) / units + 1; }
+
+DecodeShape shape_of(const cqa_cache* c, int T) {
+  DecodeShape sh;
+  sh.B = c->cfg.batch;
+  sh.Hq = c->cfg.n_q_heads;
+  sh.Hkv = c->cfg.n_kv_heads;
+  sh.G = c->G;
+  sh.d = c->cfg.head_dim;
+  sh.nb = T / BLK;
+  sh.r = T - sh.nb * BLK;
+  sh.nbm = c->nbm;
+  sh.sigma = (float)(1.0 / sqrt((double)sh.d));
+  chunking(sh.B * sh.Hkv, sh.nb, &sh.chunk_blocks, &sh.nchunks);
+  return sh;
+}
+
+__global__ void fill_range_kernel(float* vr, size_t units, int d) {
+  const size_t n = units * 2 * (size_t)d;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % (2 * (size_t)d));
+    vr[i] = c < d ? INFINITY : -INFINITY;
+  }
+}
+
+// Run one launcher; when profiling, bracket it with events on `s`.
+template <class F>
+cudaError_t run_phase(cqa_cache* c, int phase, cudaStream_t s, int nlaunch, F&& fn) {
+  if (!c->prof_on || nlaunch == 0) return fn();
+  const size_t k = c->prof_phase->size();
+  const bool timed = k < c->prof_max;
+  if (timed) {
+    while (c->prof_events->size() < 2 * (k + 1)) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return cudaErrorMemoryAllocation;
+      c->prof_events->push_back(e);
+    }
+    cudaEventRecord((*c->prof_events)[2 * k], s);
+  }
+  const cudaError_t e = fn();
+  if (timed) {
+    cudaEventRecord((*c->prof_events)[2 * k + 1], s);
+    c->prof_phase->push_back(phase);
+  } else {
+    c->prof_untimed += nlaunch;
+  }
+  c->prof_launches[phase] += nlaunch;
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* cqa_error_string(int code) {
+  switch (code) {
+    case CQA_OK: return "ok";
+    case CQA_ERR_INVALID_ARG: return "invalid argument";
+    case CQA_ERR_CUDA: return "CUDA runtime error";
+    case CQA_ERR_OOM: return "out of memory";
+    case CQA_ERR_CAPACITY: return "append exceeds the cache capacity (max_ctx)";
+    case CQA_ERR_EMPTY: return "decode on an empty layer";
+  }
+  return "unknown error";
+}
+
+int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
+  if (!cfg || !out) return CQA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const cqa_config c = *cfg;
+  if (c.n_layers < 1 || c.batch < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.max_ctx < 1)
+    return CQA_ERR_INVALID_ARG;
+  if (c.head_dim != 64 && c.head_dim != 128) return CQA_ERR_INVALID_ARG;
+  if (c.n_q_heads % c.n_kv_heads) return CQA_ERR_INVALID_ARG;
+  const int G = c.n_q_heads / c.n_kv_heads;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8) || (c.head_dim == 64 && G == 8))
+    return CQA_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return CQA_ERR_CUDA;
+  if (c.device < 0 || c.device >= ndev) return CQA_ERR_INVALID_ARG;
+  const int nbm = c.max_ctx / BLK;
+  int smem_optin = 0;
+  if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device) !=
+      cudaSuccess)
+    return CQA_ERR_CUDA;
+  if (cqa::select_smem_bytes(G, nbm) > (size_t)smem_optin) return CQA_ERR_INVALID_ARG;
+
+  DeviceGuard dg(c.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+
+  cqa_cache* cc = new (std::nothrow) cqa_cache();
+  if (!cc) return CQA_ERR_OOM;
+  cc->cfg = c;
+  cc->G = G;
+  cc->nbm = nbm;
+  const int d = c.head_dim;
+  cc->st = make_strides(nbm, d, c.max_ctx);
+  const size_t units = (size_t)c.n_layers * c.batch * c.n_kv_heads;
+  const size_t hq_rows = (size_t)c.batch * c.n_q_heads;
+  const size_t max_chunks = (size_t)max_chunks_for(c.batch * c.n_kv_heads);
+
+  // one device allocation, carved into aligned pieces
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes > 0 ? bytes : 1);
+    return o;
+  };
+  const Strides& st = cc->st;
+  const size_t o_kc = take(units * st.kcodes);
+  const size_t o_ks = take(units * st.kscale * 4);
+  const size_t o_vc = take(units * st.vcodes);
+  const size_t o_vm = take(units * st.vmeta * 4);
+  const size_t o_eta = take(units * st.eta * 4);
+  const size_t o_vr = take(units * st.vrange * 4);
+  const size_t o_kr = take(units * st.res * 2);
+  const size_t o_vrs = take(units * st.res * 2);
+  const size_t ls = (size_t)nbm * BLK + BLK;
+  const size_t o_lg = take(hq_rows * ls * 4);
+  const size_t o_e8 = take(hq_rows * nbm * 4);
+  const size_t o_dl = take(hq_rows * nbm * 4);
+  const size_t o_e16 = take(hq_rows * nbm * 4);
+  const size_t o_er = take(hq_rows * 4);
+  const size_t o_ek = take(hq_rows * 4);
+  const size_t o_kst = take(hq_rows * 4);
+  const size_t o_hf = take(hq_rows);
+  const size_t o_bf = take((size_t)c.batch * c.n_kv_heads * nbm);
+  const size_t o_dn = take(hq_rows);
+  const size_t o_po = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * d * 4);
+  const size_t o_ps = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
+  void* base = nullptr;
+  if (cudaMalloc(&base, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete cc;
+    return CQA_ERR_OOM;
+  }
+  cc->dev_block = base;
+  char* bp = (char*)base;
+  cc->t.kcodes = (int8_t*)(bp + o_kc);
+  cc->t.kscale = (float*)(bp + o_ks);
+  cc->t.vcodes = (uint8_t*)(bp + o_vc);
+  cc->t.vmeta = (float*)(bp + o_vm);
+  cc->t.eta = (float*)(bp + o_eta);
+  cc->t.vrange = (float*)(bp + o_vr);
+  cc->t.kres = (__half*)(bp + o_kr);
+  cc->t.vres = (__half*)(bp + o_vrs);
+  cc->sc.logits = (float*)(bp + o_lg);
+  cc->sc.ell8 = (float*)(bp + o_e8);
+  cc->sc.delta = (float*)(bp + o_dl);
+  cc->sc.ell16 = (float*)(bp + o_e16);
+  cc->sc.ell_res = (float*)(bp + o_er);
+  cc->sc.ekey = (float*)(bp + o_ek);
+  cc->sc.kstar = (int32_t*)(bp + o_kst);
+  cc->sc.hflags = (uint8_t*)(bp + o_hf);
+  cc->sc.bflags = (uint8_t*)(bp + o_bf);
+  cc->sc.dense = (uint8_t*)(bp + o_dn);
+  cc->sc.part_o = (float*)(bp + o_po);
+  cc->sc.part_s = (float*)(bp + o_ps);
+  cc->sc.ls = ls;
+  cc->sc.max_chunks = (int)max_chunks;
+
+  if (cudaMemset(base, 0, off) != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+  fill_range_kernel<<<256, 256>>>(cc->t.vrange, units, d);
+  if (cudaGetLastError() != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+
+  cc->tier2_bytes = units * st.tier2 * 2;
+  if (cudaHostAlloc(&cc->k2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
+          cudaSuccess ||
+      cudaHostAlloc(&cc->v2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    cqa_cache_destroy(cc);
+    return CQA_ERR_OOM;
+  }
+  void* kd = nullptr;
+  void* vd = nullptr;
+  if (cudaHostGetDevicePointer(&kd, cc->k2_host, 0) != cudaSuccess ||
+      cudaHostGetDevicePointer(&vd, cc->v2_host, 0) != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+  cc->t.k2 = (__half*)kd;
+  cc->t.v2 = (__half*)vd;
+
+  cc->len = (int32_t*)calloc((size_t)c.n_layers, sizeof(int32_t));
+  if (!cc->len) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_OOM;
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+  *out = cc;
+  return CQA_OK;
+}
+
+int cqa_cache_destroy(cqa_cache* cc) {
+  if (!cc) return CQA_OK;
+  int rc = CQA_OK;
+  {
+    DeviceGuard dg(cc->cfg.device);
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = CQA_ERR_CUDA;
+    if (cc->dev_block) cudaFree(cc->dev_block);
+    if (cc->k2_host) cudaFreeHost(cc->k2_host);
+    if (cc->v2_host) cudaFreeHost(cc->v2_host);
+    if (cc->prof_events)
+      for (cudaEvent_t ev : *cc->prof_events) cudaEventDestroy(ev);
+  }
+  delete cc->prof_events;
+  delete cc->prof_phase;
+  free(cc->len);
+  delete cc;
+  return rc;
+}
+
+int cqa_cache_length(const cqa_cache* cc, int layer, int32_t* out_len) {
+  if (!cc || !out_len || layer < 0 || layer >= cc->cfg.n_layers) return CQA_ERR_INVALID_ARG;
+  *out_len = cc->len[layer];
+  return CQA_OK;
+}
+
+int cqa_quantize_append(cqa_cache* cc, int layer, const void* k, const void* v, int n_new,
+                        void* stream) {
+  if (!cc || layer < 0 || layer >= cc->cfg.n_layers || n_new < 0) return CQA_ERR_INVALID_ARG;
+  if (n_new == 0) return CQA_OK;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return CQA_ERR_INVALID_ARG;
+  const int T_old = cc->len[layer];
+  if ((long long)T_old + n_new > cc->cfg.max_ctx) return CQA_ERR_CAPACITY;
+  const int T_new = T_old + n_new;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int B = cc->cfg.batch, Hkv = cc->cfg.n_kv_heads, d = cc->cfg.head_dim;
+  const int unit0 = layer * B * Hkv;
+  const int nb_old = T_old / BLK, nb_new = T_new / BLK;
+  const __half* kh = (const __half*)k;
+  const __half* vh = (const __half*)v;
+  cudaError_t e = run_phase(cc, CQA_PHASE_APPEND_SEAL, s, nb_new > nb_old ? 1 : 0, [&] {
+    return launch_seal(cc->t, cc->st, unit0, B, Hkv, d, kh, vh, T_old, n_new, nb_old, nb_new, s);
+  });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_APPEND_TAIL, s, 1, [&] {
+      return launch_append_tail(cc->t, cc->st, unit0, B, Hkv, d, kh, vh, T_old, n_new, nb_new, s);
+    });
+  if (e != cudaSuccess) return CQA_ERR_CUDA;
+  cc->len[layer] = T_new;
+  return CQA_OK;
+}
+
+static int copy_trace(cqa_cache* cc, const DecodeShape& sh, const cqa_trace* tr, cudaStream_t s) {
+  const size_t rows = (size_t)sh.B * sh.Hq;
+  cudaError_t e = cudaSuccess;
+  auto cp2 = [&](void* dst, const void* src, size_t elem, size_t width, size_t pitch,
+                 size_t nrows) {
+    if (!dst || e != cudaSuccess || width == 0) return;
+    e = cudaMemcpy2DAsync(dst, width * elem, src, pitch * elem, width * elem, nrows,
+                          cudaMemcpyDeviceToDevice, s);
+  };
+  cp2(tr->kstar, cc->sc.kstar, 4, rows, rows, 1);
+  cp2(tr->head_flags, cc->sc.hflags, 1, rows, rows, 1);
+  cp2(tr->ell_res, cc->sc.ell_res, 4, rows, rows, 1);
+  cp2(tr->block_flags, cc->sc.bflags, 1, sh.nb, sh.nbm, (size_t)sh.B * sh.Hkv);
+  cp2(tr->ell8, cc->sc.ell8, 4, sh.nb, sh.nbm, rows);
+  cp2(tr->ell16, cc->sc.ell16, 4, sh.nb, sh.nbm, rows);
+  cp2(tr->delta, cc->sc.delta, 4, sh.nb, sh.nbm, rows);
+  return e == cudaSuccess ? CQA_OK : CQA_ERR_CUDA;
+}
+
+int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th, float* out,
+               float* e_key, float* e_val, uint8_t* rung, const cqa_trace* trace, void* stream) {
+  if (!cc || layer < 0 || layer >= cc->cfg.n_layers || !q || !th || !out || !e_key || !e_val ||
+      !rung)
+    return CQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return CQA_ERR_INVALID_ARG;
+  const cqa_thresholds tv = *th;
+  if (!(tv.tau_cov >= 0.f) || tv.max_expand < 0 || tv.rank_r < 0 || isnan(tv.eps_key) ||
+      isnan(tv.v_tol) || isnan(tv.eps_val) || isnan(tv.layer_dense_frac))
+    return CQA_ERR_INVALID_ARG;
+  const int T = cc->len[layer];
+  if (T == 0) return CQA_ERR_EMPTY;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const DecodeShape sh = shape_of(cc, T);
+  if (sh.nchunks > cc->sc.max_chunks) return CQA_ERR_INVALID_ARG;
+  const int unit0 = layer * sh.B * sh.Hkv;
+  double need = ceil((double)tv.layer_dense_frac * sh.Hq);
+  if (need < 0) need = 0;
+  const int need_dense = need > 1e9 ? 1000000000 : (int)need;
+  const __half* qh = (const __half*)q;
+  cudaError_t e = run_phase(cc, CQA_PHASE_SCORE, s, 1,
+                            [&] { return launch_score(cc->t, cc->st, unit0, sh, qh, cc->sc, s); });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_SELECT, s, 1,
+                  [&] { return launch_select(cc->t, cc->st, unit0, sh, tv, cc->sc, s); });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_ATTEND, s, 1,
+                  [&] { return launch_attend(cc->t, cc->st, unit0, sh, qh, cc->sc, 0, s); });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_COMBINE, s, 1, [&] {
+      return launch_combine(sh, tv, need_dense, cc->sc, out, e_key, e_val, rung, s);
+    });
+  if (e == cudaSuccess && !tv.naive) {
+    e = run_phase(cc, CQA_PHASE_DENSE_ATTEND, s, 1,
+                  [&] { return launch_attend(cc->t, cc->st, unit0, sh, qh, cc->sc, 1, s); });
+    if (e == cudaSuccess)
+      e = run_phase(cc, CQA_PHASE_DENSE_COMBINE, s, 1, [&] {
+        return launch_dense_combine(sh, cc->sc, 0, out, e_key, e_val, rung, s);
+      });
+  }
+  if (e != cudaSuccess) return CQA_ERR_CUDA;
+  if (trace) return copy_trace(cc, sh, trace, s);
+  return CQA_OK;
+}
+
+int cqa_dense_reference(cqa_cache* cc, int layer, const void* q, float* out, void* stream) {
+  if (!cc || layer < 0 || layer >= cc->cfg.n_layers || !q || !out) return CQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return CQA_ERR_INVALID_ARG;
+  const int T = cc->len[layer];
+  if (T == 0) return CQA_ERR_EMPTY;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const DecodeShape sh = shape_of(cc, T);
+  const int unit0 = layer * sh.B * sh.Hkv;
+  cudaError_t e = run_phase(cc, CQA_PHASE_DENSE_ATTEND, s, 1, [&] {
+    return launch_attend(cc->t, cc->st, unit0, sh, (const __half*)q, cc->sc, 2, s);
+  });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_DENSE_COMBINE, s, 1, [&] {
+      return launch_dense_combine(sh, cc->sc, 1, out, nullptr, nullptr, nullptr, s);
+    });
+  return e == cudaSuccess ? CQA_OK : CQA_ERR_CUDA;
+}
+
+int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t bytes) {
+  if (!cc || layer < 0 || layer >= cc->cfg.n_layers) return CQA_ERR_INVALID_ARG;
+  const int B = cc->cfg.batch, Hkv = cc->cfg.n_kv_heads, d = cc->cfg.head_dim;
+  const int T = cc->len[layer];
+  const int nb = T / BLK, r = T - nb * BLK;
+  const size_t units = (size_t)B * Hkv;
+  const size_t unit0 = (size_t)layer * units;
+  const Strides& st = cc->st;
+  const char* srcs[2] = {nullptr, nullptr};
+  size_t per_unit = 0, stride = 0;  // bytes
+  bool host_src = false;
+  int parts = 1;
+  switch (what) {
+    case CQA_EXPORT_KCODES: srcs[0] = (const char*)cc->t.kcodes; per_unit = (size_t)nb * BLK * d; stride = st.kcodes; break;
+    case CQA_EXPORT_KSCALE: srcs[0] = (const char*)cc->t.kscale; per_unit = (size_t)nb * d * 4; stride = st.kscale * 4; break;
+    case CQA_EXPORT_VCODES: srcs[0] = (const char*)cc->t.vcodes; per_unit = (size_t)nb * BLK * d / 2; stride = st.vcodes; break;
+    case CQA_EXPORT_VMETA: srcs[0] = (const char*)cc->t.vmeta; per_unit = (size_t)nb * BLK * (d / VG) * 8; stride = st.vmeta * 4; break;
+    case CQA_EXPORT_ETA: srcs[0] = (const char*)cc->t.eta; per_unit = (size_t)nb * 4; stride = st.eta * 4; break;
+    case CQA_EXPORT_VRANGE: srcs[0] = (const char*)cc->t.vrange; per_unit = (size_t)2 * d * 4; stride = st.vrange * 4; break;
+    case CQA_EXPORT_RESIDUAL:
+      srcs[0] = (const char*)cc->t.kres; srcs[1] = (const char*)cc->t.vres;
+      per_unit = (size_t)r * d * 2; stride = st.res * 2; parts = 2;
+      break;
+    case CQA_EXPORT_TIER2:
+      srcs[0] = (const char*)cc->k2_host; srcs[1] = (const char*)cc->v2_host;
+      per_unit = (size_t)T * d * 2; stride = st.tier2 * 2; parts = 2;
+      host_src = true;
+      break;
+    default: return CQA_ERR_INVALID_ARG;
+  }
+  const size_t total = units * parts * per_unit;
+  if (!dst && bytes == 0) return (int64_t)total;
+  if (!dst || bytes != total) return CQA_ERR_INVALID_ARG;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok || cudaDeviceSynchronize() != cudaSuccess) return CQA_ERR_CUDA;
+  char* out = (char*)dst;
+  for (size_t uu = 0; uu < units; ++uu) {
+    for (int p = 0; p < parts; ++p) {
+      const char* sp = srcs[p] + (unit0 + uu) * stride;
+      char* dp = out + (uu * parts + p) * per_unit;
+      if (per_unit == 0) continue;
+      if (host_src) {
+        memcpy(dp, sp, per_unit);
+      } else if (cudaMemcpy(dp, sp, per_unit, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        return CQA_ERR_CUDA;
+      }
+    }
+  }
+  return (int64_t)total;
+}
+
+int cqa_profile_begin(cqa_cache* cc, int max_launches) {
+  if (!cc || max_launches < 0) return CQA_ERR_INVALID_ARG;
+  if (!cc->prof_events) {
+    cc->prof_events = new (std::nothrow) std::vector<cudaEvent_t>();
+    cc->prof_phase = new (std::nothrow) std::vector<int>();
+    if (!cc->prof_events || !cc->prof_phase) return CQA_ERR_OOM;
+  }
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  cc->prof_phase->clear();
+  cc->prof_max = (size_t)max_launches;
+  cc->prof_untimed = 0;
+  for (int i = 0; i < CQA_PHASE_COUNT; ++i) cc->prof_launches[i] = 0;
+  cc->prof_on = true;
+  return CQA_OK;
+}
+
+int cqa_profile_end(cqa_cache* cc, double* ms, int64_t* launches) {
+  if (!cc || !cc->prof_on) return CQA_ERR_INVALID_ARG;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  cc->prof_on = false;
+  double acc[CQA_PHASE_COUNT] = {0};
+  for (size_t k = 0; k < cc->prof_phase->size(); ++k) {
+    cudaEvent_t a = (*cc->prof_events)[2 * k], b = (*cc->prof_events)[2 * k + 1];
+    if (cudaEventSynchronize(b) != cudaSuccess) return CQA_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, a, b) != cudaSuccess) return CQA_ERR_CUDA;
+    acc[(*cc->prof_phase)[k]] += t;
+  }
+  for (int i = 0; i < CQA_PHASE_COUNT; ++i) {
+    if (ms) ms[i] = acc[i];
+    if (launches) launches[i] = cc->prof_launches[i];
+  }
+  return (int)(cc->prof_untimed > 0x7fffffff ? 0x7fffffff : cc->prof_untimed);
+}
+
+}  // extern "C"

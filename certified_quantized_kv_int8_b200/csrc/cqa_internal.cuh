@@ -1,0 +1,113 @@
+// Internal declarations shared by the CUDA sources of libcqa.so.
+//
+// Data layout in device memory (Tier 1) for one unit u = (layer, batch row,
+// kv head), nbm = max_ctx / 64 block slots, d = head_dim:
+//   kcodes int8  [nbm][64][d]        token-major: one 16-byte load = 16 channels
+//   kscale fp32  [nbm][d]            per (block, channel) key scale
+//   vcodes uint8 [nbm][64][d/2]      INT4 pairs, channel 2j in the low nibble
+//   vmeta  fp32  [nbm][64][d/32][2]  per (token, group): scale, offset
+//   eta    fp32  [nbm]               per-block max INT4 reconstruction error
+//   vrange fp32  [2][d]              running per-channel value min and max
+//   kres, vres fp16 [64][d]          the residual (unsealed) block, exact
+// Tier 2 (pinned host, device-mapped): k2, v2 fp16 [max_ctx][d] per unit.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cqa.h"
+
+namespace cqa {
+
+constexpr int BLK = 64;  // tokens per block
+constexpr int VG = 32;   // channels per INT4 value group
+
+// bits of the per-block flag byte
+constexpr uint8_t BF_KEY = 1;  // FP16 keys promoted
+constexpr uint8_t BF_VAL = 2;  // FP16 values promoted
+// bits of the per-head flag byte
+constexpr uint8_t HF_WIDENED = 1;
+constexpr uint8_t HF_VALUE = 2;
+constexpr uint8_t HF_KEYFAIL = 4;
+constexpr uint8_t HF_RANKFAIL = 8;
+constexpr uint8_t HF_VALFAIL = 16;
+
+struct Tier1 {
+  int8_t* kcodes;
+  float* kscale;
+  uint8_t* vcodes;
+  float* vmeta;
+  float* eta;
+  float* vrange;
+  __half* kres;
+  __half* vres;
+  __half* k2;  // device view of Tier 2 keys
+  __half* v2;  // device view of Tier 2 values
+};
+
+// element strides per unit
+struct Strides {
+  size_t kcodes, kscale, vcodes, vmeta, eta, vrange, res, tier2;
+};
+
+inline Strides make_strides(int nbm, int d, int max_ctx) {
+  Strides s;
+  s.kcodes = (size_t)nbm * BLK * d;
+  s.kscale = (size_t)nbm * d;
+  s.vcodes = (size_t)nbm * BLK * d / 2;
+  s.vmeta = (size_t)nbm * BLK * (d / VG) * 2;
+  s.eta = (size_t)nbm;
+  s.vrange = (size_t)2 * d;
+  s.res = (size_t)BLK * d;
+  s.tier2 = (size_t)max_ctx * d;
+  return s;
+}
+
+// Scratch of one decode call (device), sized for nbm blocks.
+struct Scratch {
+  float* logits;     // [B][Hq][ls]  INT8 logits (sealed) + exact residual logits
+  float* ell8;       // [B][Hq][nbm]
+  float* delta;      // [B][Hq][nbm]
+  float* ell16;      // [B][Hq][nbm]
+  float* ell_res;    // [B][Hq]
+  float* ekey;       // [B][Hq]
+  int32_t* kstar;    // [B][Hq]
+  uint8_t* hflags;   // [B][Hq]
+  uint8_t* bflags;   // [B][Hkv][nbm]
+  uint8_t* dense;    // [B][Hq] 0, 3 or 4
+  float* part_o;     // [B*Hkv][max_chunks][G][d]
+  float* part_s;     // [B*Hkv][max_chunks][G][3]  (m, l, eta mass)
+  size_t ls;         // logits row stride = nbm * 64 + 64
+  int max_chunks;
+};
+
+struct DecodeShape {
+  int B, Hq, Hkv, G, d, nb, r, nbm, nchunks, chunk_blocks;
+  float sigma;
+};
+
+// ---- launchers (each returns the launch error, cudaSuccess on success) ----
+cudaError_t launch_seal(const Tier1& t, const Strides& st, int layer_unit0, int B, int Hkv, int d,
+                        const __half* knew, const __half* vnew, int T_old, int n_new, int nb_old,
+                        int nb_new, cudaStream_t s);
+cudaError_t launch_append_tail(const Tier1& t, const Strides& st, int layer_unit0, int B, int Hkv,
+                               int d, const __half* knew, const __half* vnew, int T_old,
+                               int n_new, int nb_new, cudaStream_t s);
+cudaError_t launch_score(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
+                         const __half* q, const Scratch& sc, cudaStream_t s);
+cudaError_t launch_select(const Tier1& t, const Strides& st, int layer_unit0,
+                          const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
+                          cudaStream_t s);
+// mode 0: certified (block flags decide), 1: dense for flagged heads, 2: dense for all
+cudaError_t launch_attend(const Tier1& t, const Strides& st, int layer_unit0,
+                          const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
+                          cudaStream_t s);
+cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
+                           const Scratch& sc, float* out, float* e_key, float* e_val,
+                           uint8_t* rung, cudaStream_t s);
+cudaError_t launch_dense_combine(const DecodeShape& sh, const Scratch& sc, int all_heads,
+                                 float* out, float* e_key, float* e_val, uint8_t* rung,
+                                 cudaStream_t s);
+
+}  // namespace cqa

@@ -1,0 +1,203 @@
+/*
+ * cqa.h — C ABI of the certified quantized KV-cache decode-attention library
+ * (libcqa.so, CUDA for sm_100a).
+ *
+ * The library implements the decode-step hot path of *Runtime-Certified
+ * Bounded-Error Quantized Attention* (gist.science summary of paper
+ * 2605.20868, technical summary):
+ *   - Methodology §1 "Tiered storage with deterministic fallback": Tier 1 in
+ *     device memory (per-channel INT8 keys, per-group INT4 values, their
+ *     scales/offsets, per-block error annotations eta_b); Tier 2 in pinned
+ *     host RAM (the FP16 originals).
+ *   - Methodology §2 "Two-term error decomposition": per head and step, a key
+ *     bound E_key (total-variation distance of the softmax, from the per-token
+ *     score perturbation Delta) and a value bound E_val (attention mass times
+ *     eta_b), computed from Tier-1 quantities only.
+ *   - Methodology §3 "Adaptive precision and fallback ladder": an INT8 scoring
+ *     pass, promotion of the top-K* blocks covering tau_cov of the estimated
+ *     mass to FP16 keys paged from Tier 2, a block-ranking consistency check,
+ *     and the four rungs (widen coverage, FP16 values, per-head dense,
+ *     whole-layer dense).
+ *
+ * Conventions for every entry point:
+ *   - Return value: CQA_OK (0) or a negative CQA_ERR_* code; cqa_error_string
+ *     names it.  On an argument error nothing is launched and no output is
+ *     written.  CQA_ERR_CUDA reports a failed CUDA call; the cache may then be
+ *     in an unspecified state and should be destroyed.
+ *   - Device pointers are plain CUDA device addresses (cudaMalloc or any
+ *     allocator of the same device); `stream` is a cudaStream_t passed as
+ *     void* (NULL = the legacy default stream).  Calls enqueue work on
+ *     `stream` and return; results are valid once the stream has synchronised.
+ *   - Ownership: the caller owns every pointer it passes; the library owns
+ *     both tiers and all scratch memory held by a cqa_cache.
+ *   - Threading: a cache may be used by one host thread at a time, and two
+ *     calls on one cache must not overlap on the GPU (use one stream, or order
+ *     the streams).
+ *   - Layouts are row-major C arrays; "fp16" is IEEE binary16.
+ */
+#ifndef CQA_H
+#define CQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  CQA_OK = 0,
+  CQA_ERR_INVALID_ARG = -1, /* null pointer, bad shape, layer out of range, ... */
+  CQA_ERR_CUDA = -2,        /* a CUDA runtime call failed */
+  CQA_ERR_OOM = -3,         /* device or pinned-host allocation failed */
+  CQA_ERR_CAPACITY = -4,    /* the append would exceed max_ctx */
+  CQA_ERR_EMPTY = -5        /* decode on a layer that holds no token */
+};
+
+typedef struct cqa_cache cqa_cache; /* opaque */
+
+/* Shape of one cache: every layer holds `batch` sequences of equal length. */
+typedef struct cqa_config {
+  int32_t n_layers;
+  int32_t batch;
+  int32_t n_q_heads;  /* query heads; query head h reads kv head h / (n_q_heads / n_kv_heads) */
+  int32_t n_kv_heads; /* must divide n_q_heads; n_q_heads / n_kv_heads in {1, 2, 4, 8} */
+  int32_t head_dim;   /* 64 or 128 */
+  int32_t max_ctx;    /* token capacity per (layer, batch row), >= 1 */
+  int32_t device;     /* CUDA device ordinal the cache lives on */
+} cqa_config;
+
+/* Runtime thresholds of one decode call (Methodology §3).  tau_cov and v_tol
+ * are named by the method; the other fields are this library's readings of
+ * triggers the method leaves unstated. */
+typedef struct cqa_thresholds {
+  float tau_cov;          /* promote the fewest blocks whose INT8-estimated mass, plus the
+                             exact residual block, reaches tau_cov; >= 1 promotes all */
+  float eps_key;          /* rung 1: widen K* (doubling) while E_key > eps_key ... */
+  int32_t max_expand;     /* ... at most max_expand times; still above -> rung 3 */
+  float v_tol;            /* rung 2: FP16 values for block b if some head's
+                             m8_b * eta_b > v_tol (m8 = INT8-estimated block mass) */
+  int32_t rank_r;         /* rank check: ordered top-min(rank_r, |P|) promoted blocks by
+                             INT8 and by FP16 log-mass must agree, else rung 3 */
+  float eps_val;          /* rung 3 also when E_val > eps_val (+inf disables) */
+  float layer_dense_frac; /* rung 4 when >= ceil(layer_dense_frac * n_q_heads) heads of a
+                             (layer, batch row) took rung 3 */
+  int32_t naive;          /* 1: certification off (no promotion, no ladder; bounds still
+                             reported), 0: certified */
+} cqa_thresholds;
+
+/* Optional per-call diagnostics, all device pointers, any may be NULL.
+ * nb = number of sealed 64-token blocks of the layer (length / 64). */
+typedef struct cqa_trace {
+  int32_t* kstar;       /* [batch][n_q_heads] final K* after widening */
+  uint8_t* block_flags; /* [batch][n_kv_heads][nb]: bit0 key promoted, bit1 value promoted */
+  float* ell8;          /* [batch][n_q_heads][nb] INT8 block log-mass (natural log) */
+  float* ell16;         /* [batch][n_q_heads][nb] FP16 block log-mass, promoted blocks only */
+  float* delta;         /* [batch][n_q_heads][nb] per-token score perturbation bound Delta */
+  uint8_t* head_flags;  /* [batch][n_q_heads]: bit0 widened, bit1 value promotion,
+                           bit2 E_key fail, bit3 rank fail, bit4 E_val fail */
+  float* ell_res;       /* [batch][n_q_heads] log-mass of the exact residual block (-inf if empty) */
+} cqa_trace;
+
+/* Allocate both tiers for `cfg` on cfg->device: Tier 1 and scratch in device
+ * memory, Tier 2 (n_layers * batch * n_kv_heads * max_ctx * head_dim * 2 fp16)
+ * in pinned, device-mapped host memory.  *out receives the handle. */
+int cqa_cache_create(const cqa_config* cfg, cqa_cache** out);
+
+/* Free everything the cache owns (synchronises the device first).  NULL is a no-op. */
+int cqa_cache_destroy(cqa_cache* cache);
+
+/* Tokens currently held by `layer` (host-side counter; no synchronisation). */
+int cqa_cache_length(const cqa_cache* cache, int layer, int32_t* out_len);
+
+/* Append n_new tokens to every batch row of `layer` (Methodology §1).
+ * k_fp16, v_fp16: device fp16 [batch][n_kv_heads][n_new][head_dim].
+ * Every complete 64-token block is sealed: keys -> symmetric INT8 with one
+ * fp32 scale per (block, channel) (s = amax/127, code = round-half-even(k/s)),
+ * values -> asymmetric INT4 per (token, 32 channels) (z = min,
+ * s = (max-min)/15), eta_b = max |v - (s*code + z)| over the block; the newest
+ * length % 64 tokens stay exact in FP16 (the residual block).  All appended
+ * tokens are also written to Tier 2.  The encoding of a block depends only on
+ * its tokens, so appending in any chunking gives the same cache.
+ * CQA_ERR_CAPACITY if length + n_new > max_ctx.  n_new = 0 is a no-op. */
+int cqa_quantize_append(cqa_cache* cache, int layer, const void* k_fp16, const void* v_fp16,
+                        int n_new, void* stream);
+
+/* One certified decode step of `layer` for all batch rows (Methodology §2-§3).
+ * q_fp16: device fp16 [batch][n_q_heads][head_dim].
+ * Outputs (device): out fp32 [batch][n_q_heads][head_dim]; e_key, e_val fp32
+ * [batch][n_q_heads]; rung uint8 [batch][n_q_heads] = highest rung reached:
+ * 0 certified as selected, 1 coverage widened, 2 FP16 values promoted,
+ * 3 per-head dense, 4 whole-layer dense.  Dense heads return exact attention
+ * over the FP16 originals with e_key = e_val = 0.  For the other heads
+ * max_c |out - O_dense| <= R_V * e_key + e_val, R_V = max_c (vmax_c - vmin_c)
+ * of the head's kv head (exported by cqa_debug_export).
+ * th: host pointer.  trace: host pointer to a cqa_trace, or NULL.
+ * CQA_ERR_EMPTY if the layer holds no token. */
+int cqa_decode(cqa_cache* cache, int layer, const void* q_fp16, const cqa_thresholds* th,
+               float* out, float* e_key, float* e_val, uint8_t* rung, const cqa_trace* trace,
+               void* stream);
+
+/* Exact attention softmax(q K^T / sqrt(head_dim)) V of `layer` over the FP16
+ * originals (Tier 2 plus the residual block), fp32 accumulation: the O_dense
+ * the fallback ladder returns.  q_fp16 and out as in cqa_decode. */
+int cqa_dense_reference(cqa_cache* cache, int layer, const void* q_fp16, float* out, void* stream);
+
+/* Copy one Tier-1 array of `layer` to host memory (synchronous; for tests and
+ * inspection).  `what` selects the array, laid out as stated, with nb the
+ * layer's sealed block count and d = head_dim:
+ *   CQA_EXPORT_KCODES   int8  [batch][n_kv_heads][nb][64][d]
+ *   CQA_EXPORT_KSCALE   fp32  [batch][n_kv_heads][nb][d]
+ *   CQA_EXPORT_VCODES   uint8 [batch][n_kv_heads][nb][64][d/2]  (channel 2j low nibble)
+ *   CQA_EXPORT_VMETA    fp32  [batch][n_kv_heads][nb][64][d/32][2]  (scale, offset)
+ *   CQA_EXPORT_ETA      fp32  [batch][n_kv_heads][nb]
+ *   CQA_EXPORT_VRANGE   fp32  [batch][n_kv_heads][2][d]  (vmin, vmax over all tokens)
+ *   CQA_EXPORT_RESIDUAL fp16  [batch][n_kv_heads][2][length % 64][d]  (keys, values)
+ *   CQA_EXPORT_TIER2    fp16  [batch][n_kv_heads][2][length][d]  (keys, values)
+ * `bytes` must equal the array's size (CQA_ERR_INVALID_ARG otherwise);
+ * cqa_debug_export(cache, layer, what, NULL, 0) returns that size instead
+ * (as a non-negative value, or a negative error). */
+enum {
+  CQA_EXPORT_KCODES = 0,
+  CQA_EXPORT_KSCALE = 1,
+  CQA_EXPORT_VCODES = 2,
+  CQA_EXPORT_VMETA = 3,
+  CQA_EXPORT_ETA = 4,
+  CQA_EXPORT_VRANGE = 5,
+  CQA_EXPORT_RESIDUAL = 6,
+  CQA_EXPORT_TIER2 = 7
+};
+int64_t cqa_debug_export(cqa_cache* cache, int layer, int what, void* host_dst, size_t bytes);
+
+/* Per-phase device time of the library's kernels (tracing).  Between
+ * cqa_profile_begin and cqa_profile_end, every kernel the cache launches is
+ * bracketed by two CUDA events recorded on the call's stream; end waits for
+ * them and reports, per phase, the summed event time in milliseconds and the
+ * number of kernel launches.  Phases: */
+enum {
+  CQA_PHASE_APPEND_SEAL = 0,   /* sealing complete blocks into Tier 1 */
+  CQA_PHASE_APPEND_TAIL = 1,   /* Tier-2 copy, residual block, value ranges */
+  CQA_PHASE_SCORE = 2,         /* INT8 scoring pass */
+  CQA_PHASE_SELECT = 3,        /* coverage selection, E_key, rungs 1-2 */
+  CQA_PHASE_ATTEND = 4,        /* split-K attention with fused promotion */
+  CQA_PHASE_COMBINE = 5,       /* combine, E_val, rank check, rungs 3-4 */
+  CQA_PHASE_DENSE_ATTEND = 6,  /* exact attention of dense-fallback heads */
+  CQA_PHASE_DENSE_COMBINE = 7, /* combine of the dense fallback */
+  CQA_PHASE_COUNT = 8
+};
+/* Start (or restart) profiling; max_launches bounds the recorded launches
+ * (further launches are counted but not timed). */
+int cqa_profile_begin(cqa_cache* cache, int max_launches);
+/* Stop profiling.  ms[CQA_PHASE_COUNT] and launches[CQA_PHASE_COUNT] are host
+ * arrays (either may be NULL).  Returns the number of launches left untimed
+ * (>= 0) or a negative error. */
+int cqa_profile_end(cqa_cache* cache, double* ms, int64_t* launches);
+
+/* Static description of an error code. */
+const char* cqa_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CQA_H */

@@ -1,0 +1,158 @@
+"""GPU parity of the certified decode step and of the dense reference against the oracle."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic_kv as sk
+from tests.gpu_util import (OUT_TOL, TieLog, compare_decode, fill_cache, oracle_thresholds,
+                            oracle_units, row, run_decode)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cqa():
+    import certified_quantized_kv_int8_b200 as m
+    from certified_quantized_kv_int8_b200.build import build
+    build()
+    m.load_library()
+    return m
+
+
+def _check(cqa, w, ctx, th, layers=(0,), step=0, label=""):
+    from oracle import decode
+    log = TieLog()
+    with cqa.Cache(len(layers), w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx) as cache:
+        fill_cache(cache, w, list(layers), ctx)
+        for i, layer in enumerate(layers):
+            q = sk.queries(w, layer, step, "cuda")
+            res = run_decode(cache, i, q, th)
+            qc = q.cpu().numpy()
+            for b in range(w.batch):
+                units = oracle_units(w, layer, b, ctx)
+                ora = decode(qc[b], units, oracle_thresholds(th))
+                compare_decode(row(res, b), ora, oracle_thresholds(th), w.group, log,
+                               label=f"{label} layer {layer} b {b}")
+    for e in log.entries:
+        print("tie logged:", e)
+    return log
+
+
+TINY_TH = {
+    "default": {},
+    "tau0.5": dict(tau_cov=0.5),
+    "tau0.9_vtol": dict(tau_cov=0.9, v_tol=2e-3),
+    "widen": dict(tau_cov=0.3, eps_key=1e-3, max_expand=6),
+    "naive": dict(naive=True),
+    "full_promotion": dict(tau_cov=1.0, v_tol=0.0),
+    "head_dense": dict(tau_cov=0.3, eps_key=-1.0, max_expand=0),
+    "layer_dense": dict(layer_dense_frac=0.0),
+    "rank2": dict(rank_r=2, tau_cov=0.8),
+}
+
+
+@pytest.mark.parametrize("case", list(TINY_TH))
+@pytest.mark.parametrize("ctx", [1024, 1024 + 19])
+def test_decode_tiny(cqa, case, ctx):
+    w = sk.WORKLOADS["tiny"]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), **TINY_TH[case]})
+    log = _check(cqa, w, ctx, th, label=case)
+    assert len(log.entries) <= 1
+
+
+@pytest.mark.parametrize("ctx", [1, 37, 64, 65, 128 + 63])
+def test_decode_short_contexts(cqa, ctx):
+    w = sk.WORKLOADS["tiny"]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.7})
+    _check(cqa, w, ctx, th, label=f"ctx{ctx}")
+
+
+def test_decode_llama8b_8k(cqa):
+    w = sk.WORKLOADS["llama8b_8k_1layer"]
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    _check(cqa, w, w.ctx, th, label="8k")
+    th2 = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.6, "v_tol": 2e-3})
+    _check(cqa, w, w.ctx + 21, th2, label="8k-tail")
+
+
+def test_full_promotion_equals_dense_reference(cqa):
+    w = sk.WORKLOADS["llama8b_8k_1layer"]
+    from oracle import dense_attention
+    ctx = w.ctx + 9
+    with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx) as cache:
+        fill_cache(cache, w, [0], ctx)
+        q = sk.queries(w, 0, 0, "cuda")
+        dense = cache.dense_reference(0, q).cpu().numpy()
+        out, ek, ev, rung = cache.decode(0, q, cqa.Thresholds(tau_cov=1.0, v_tol=0.0, rank_r=0,
+                                                              layer_dense_frac=2.0))
+        torch.cuda.synchronize()
+        assert np.all(ek.cpu().numpy() == 0) and np.all(ev.cpu().numpy() == 0)
+        assert np.abs(out.cpu().numpy() - dense).max() <= 1e-5
+        forced = cache.decode(0, q, cqa.Thresholds(layer_dense_frac=0.0))[0].cpu().numpy()
+        assert np.array_equal(forced, dense)
+        K, V = sk.kv_layer(w, 0, 0, ctx, "cpu")
+        qc = q.cpu().numpy()[0]
+        G = w.group
+        for h in range(w.n_q_heads):
+            ref = dense_attention(qc[h:h + 1], K[0, h // G].numpy(), V[0, h // G].numpy())[0]
+            assert np.abs(dense[0, h] - ref).max() <= 1e-4
+
+
+def test_bounds_certify_the_device_output(cqa):
+    """max_c |out - O_dense| <= R_V E_key + E_val on every certified head."""
+    w = sk.WORKLOADS["llama8b_8k_1layer"]
+    ctx = w.ctx
+    with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx) as cache:
+        fill_cache(cache, w, [0], ctx)
+        q = sk.queries(w, 0, 3, "cuda")
+        for tau in (0.5, 0.9, 0.995):
+            th = cqa.Thresholds(tau_cov=tau, eps_key=1.0, rank_r=0, layer_dense_frac=2.0,
+                                v_tol=float("inf"))
+            out, ek, ev, rung = cache.decode(0, q, th)
+            dense = cache.dense_reference(0, q)
+            torch.cuda.synchronize()
+            vr = cache.export(0, 5)[0]
+            rv = (vr[:, 1] - vr[:, 0]).max(axis=1)
+            err = (out - dense).abs().amax(dim=2).cpu().numpy()[0]
+            bound = np.repeat(rv, w.group) * ek.cpu().numpy()[0] + ev.cpu().numpy()[0]
+            assert np.all(err <= bound * (1 + 1e-3) + 1e-5)
+
+
+@pytest.mark.parametrize("name,layers,ctx_extra", [
+    ("llama8b_32k_32layer_append", (0, 31), 0),
+    ("llama8b_64k_b4_t3values", (5,), 0),
+    ("llama8b_128k_needle", (17, 3), 0),
+])
+def test_decode_full_size_sampled(cqa, name, layers, ctx_extra):
+    """Full-context decode in the launch configuration of the benchmark, checked
+    against the oracle on sampled layers (every batch row and head of them)."""
+    w = sk.WORKLOADS[name]
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    log = _check(cqa, w, w.ctx + ctx_extra, th, layers=layers, label=name)
+    assert len(log.entries) <= 4
+
+
+def test_appended_steps_match_oracle(cqa):
+    """The 32K workload appends one token per layer before each decode step."""
+    from oracle import decode
+    w = sk.WORKLOADS["llama8b_32k_32layer_append"]
+    w = dataclasses.replace(w, ctx=4096, appends=8)
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    log = TieLog()
+    with cqa.Cache(1, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, w.max_ctx) as cache:
+        fill_cache(cache, w, [7], w.ctx)
+        for step in range(w.appends):
+            t = w.ctx + step
+            K, V = sk.kv_layer(w, 7, t, t + 1, "cuda")
+            cache.append(0, K, V)
+            q = sk.queries(w, 7, step, "cuda")
+            res = run_decode(cache, 0, q, th)
+            if step in (0, 5, 7):
+                units = oracle_units(w, 7, 0, t + 1)
+                ora = decode(q.cpu().numpy()[0], units, oracle_thresholds(th))
+                compare_decode(row(res, 0), ora, oracle_thresholds(th), w.group, log,
+                               label=f"step {step}")
+    assert len(log.entries) <= 1
