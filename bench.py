@@ -1,0 +1,555 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of certified quantized KV-cache attention on B200.
+
+One step = one decode step of the whole layer stack of the workload: for every
+layer, append the step's new token (workloads that append) and run the
+certified decode (INT8 scoring, coverage selection, fused FP16 promotion from
+pinned Tier 2, split-K attention with the value bound, combine, rank check,
+fallback ladder).  The line printed on rank 0 reports:
+
+  value        decode steps/s of the whole job (inputs resident on the device)
+  e2e          the same through the public API with the step's inputs copied
+               from pinned host buffers and its outputs read back every step
+  int8_int4_path  the same stack with certification off (no promotion, no
+               ladder): Tier-1 bytes per step / step time = effective KV GB/s
+  roofline     the dominant kernel of the certified step against its bound
+  roofline_hbm the INT8 scoring kernel against the measured HBM peak
+  cpu_baseline the CPU oracle on a bounded sample of the same workload
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+       python bench.py --impl reference ...   (the CPU oracle arm)
+Multi-GPU: torchrun --nproc-per-node N bench.py --gpus N: every rank runs an
+independent replica (its own sequences, seed = rank); no collective is on the
+data path, timing is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synthetic_kv as sk  # noqa: E402
+
+METRIC = "decode-attn steps/s and effective KV GB/s vs HBM peak at 8K–128K ctx"
+DEFAULT_WORKLOAD = "llama8b_32k_32layer_append"
+BLOCK = 64
+
+
+# ---------------------------------------------------------------- helpers ----
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def tier1_bytes_per_block(d: int) -> int:
+    """INT8 key codes + key scales + INT4 value codes + value scale/offset + eta_b."""
+    return BLOCK * d + 4 * d + BLOCK * d // 2 + BLOCK * (d // 32) * 8 + 4
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws: int, backend: str, timeout_s: float = 120.0):
+    if ws <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of a host float over all ranks (the timing reduction)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is None:
+        return
+    if device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+def weak_scaling_value(steps_per_rank: int, n_ranks: int, max_elapsed_s: float) -> float:
+    """Whole-job steps/s: the steps all ranks ran over the slowest rank's time."""
+    return steps_per_rank * n_ranks / max_elapsed_s
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, path: str | None = None):
+        import tempfile
+        self.index = index
+        self.proc = None
+        if path is None:
+            fd, path = tempfile.mkstemp(prefix=f"cqa_clocks{index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
+
+    def start(self):
+        d = os.path.dirname(self.path)
+        if d:
+            os.makedirs(d, exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or not parts[1].split()[0].isdigit():
+                    continue
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def h2d_probe_gbs(device, nbytes: int = 1 << 30) -> float:
+    """Pinned host -> device copy rate (the host-link peak used for promotion)."""
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    s = torch.cuda.current_stream(device)
+    best = 0.0
+    for _ in range(4):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        d.copy_(h, non_blocking=True)
+        b.record(s)
+        b.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del h, d
+    return best
+
+
+def traffic_record(kernel: str):
+    """DRAM bytes per unit from a committed ncu summary, if the kernel source is unchanged."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "certified_quantized_kv_int8_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+            return None
+    return rec
+
+
+# --------------------------------------------------------------- our arm ----
+
+def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | None:
+    import certified_quantized_kv_int8_b200 as cqa
+
+    torch.cuda.set_device(device)
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    th_naive = dataclasses.replace(th, naive=True)
+    L, B, Hq, Hkv, d = w.n_layers, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+    appends = w.appends > 0
+    n_e2e = args.e2e_steps
+    n_naive = args.steps
+    total_steps = args.warmup + args.steps + n_e2e + n_naive
+    max_ctx = w.ctx + (total_steps if appends else 0)
+    wr = dataclasses.replace(w, seed=w.seed + rank)  # independent replica per rank
+
+    cache = cqa.Cache(L, B, Hq, Hkv, d, max_ctx, device=device.index)
+    for layer in range(L):
+        K, V = sk.kv_layer(wr, layer, 0, w.ctx, device=device)
+        cache.append(layer, K, V)
+        del K, V
+    torch.cuda.synchronize(device)
+
+    # per-step inputs, resident on the device
+    def step_inputs(step):
+        qs = [sk.queries(wr, layer, step, device) for layer in range(L)]
+        kv = []
+        if appends:
+            t = w.ctx + step
+            kv = [sk.kv_layer(wr, layer, t, t + 1, device) for layer in range(L)]
+        return qs, kv
+
+    inputs = [step_inputs(s) for s in range(total_steps)]
+    outs = cache.alloc_outputs()
+    stream = torch.cuda.current_stream(device)
+
+    def run_step(s, thr):
+        qs, kv = inputs[s]
+        for layer in range(L):
+            if appends:
+                cache.append(layer, kv[layer][0], kv[layer][1], stream)
+            cache.decode(layer, qs[layer], thr, outputs=outs, stream=stream)
+
+    def timed(first, n, thr, profile=False):
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if profile:
+            cache.profile_begin(1 << 20)
+        a.record(stream)
+        for s in range(first, first + n):
+            run_step(s, thr)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        prof = cache.profile_end() if profile else None
+        barrier(dist, device)
+        return a.elapsed_time(b) * 1e-3, prof
+
+    for s in range(args.warmup):
+        run_step(s, th)
+    torch.cuda.synchronize(device)
+
+    clocks = ClockSampler(device.index, args.clocks_csv)
+    clocks.start()
+    elapsed, prof = timed(args.warmup, args.steps, th, profile=True)
+    clk = clocks.stop()
+    t_max = max_over_ranks(elapsed, dist, device)
+    value = weak_scaling_value(args.steps, ws, t_max)
+    phase_ms, phase_n, untimed = prof
+
+    # census of the decisions (untimed, on the state after the timed steps)
+    census = dict(blocks=0, key_promoted=0, value_promoted=0, heads=0,
+                  rungs=[0, 0, 0, 0, 0])
+    for layer in range(L):
+        tr = cache.alloc_trace(layer)
+        o = cache.alloc_outputs()
+        cache.decode(layer, inputs[args.warmup + args.steps - 1][0][layer], th, outputs=o,
+                     trace=tr)
+        torch.cuda.synchronize(device)
+        bf = tr["block_flags"].cpu().numpy()
+        nb = cache.length(layer) // BLOCK
+        bf = bf[..., :nb]
+        census["blocks"] += int(bf.size)
+        census["key_promoted"] += int((bf & 1).astype(bool).sum())
+        census["value_promoted"] += int((bf & 2).astype(bool).sum())
+        rg = o[3].cpu().numpy().ravel()
+        census["heads"] += int(rg.size)
+        for r in range(5):
+            census["rungs"][r] += int((rg == r).sum())
+
+    # end to end through the public API: host inputs in, host results out, every step
+    e2e = None
+    if n_e2e > 0:
+        first = args.warmup + args.steps
+        hq = [[x.cpu().pin_memory() for x in inputs[s][0]] for s in range(first, first + n_e2e)]
+        hkv = [[(k.cpu().pin_memory(), v.cpu().pin_memory()) for k, v in inputs[s][1]]
+               for s in range(first, first + n_e2e)]
+        dq = [torch.empty_like(x) for x in inputs[0][0]]
+        dkv = [(torch.empty_like(k), torch.empty_like(v)) for k, v in inputs[0][1]]
+        ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(x.numel() * x.element_size() for x in hq[0])
+        h2d += sum(k.numel() * k.element_size() * 2 for k, _ in hkv[0])
+        d2h = L * sum(t.numel() * t.element_size() for t in outs)
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n_e2e):
+            for layer in range(L):
+                dq[layer].copy_(hq[i][layer], non_blocking=True)
+                if appends:
+                    dkv[layer][0].copy_(hkv[i][layer][0], non_blocking=True)
+                    dkv[layer][1].copy_(hkv[i][layer][1], non_blocking=True)
+                    cache.append(layer, dkv[layer][0], dkv[layer][1], stream)
+                cache.decode(layer, dq[layer], th, outputs=outs, stream=stream)
+                for h_, d_ in zip(ho, outs):
+                    h_.copy_(d_, non_blocking=True)
+            stream.synchronize()  # the step's results are on the host
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e_el = max_over_ranks(a.elapsed_time(b) * 1e-3, dist, device)
+        e2e = {"value": weak_scaling_value(n_e2e, ws, e_el), "unit": "steps/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+
+    # the INT8/INT4 path alone (certification off): effective KV GB/s
+    first = args.warmup + args.steps + n_e2e
+    n_el, nprof = timed(first, n_naive, th_naive, profile=True)
+    n_max = max_over_ranks(n_el, dist, device)
+    nb_total = sum(cache.length(layer) // BLOCK for layer in range(L))
+    t1_bytes = nb_total * B * Hkv * tier1_bytes_per_block(d)  # per step (lengths at the end)
+    peaks = measured_peaks()
+    kv_gbs = t1_bytes * n_naive / n_max / 1e9 * ws
+
+    h2d_peak = h2d_probe_gbs(device)
+
+    # dominant kernel of the certified step
+    n_steps = args.steps
+    att_ms = phase_ms["attend"] / max(1, phase_n["attend"])
+    ctx_mid = cache.length(0)
+    nb_mid = ctx_mid // BLOCK
+    frac_k = census["key_promoted"] / max(1, census["blocks"])
+    frac_v = census["value_promoted"] / max(1, census["blocks"])
+    per_block_h2d = BLOCK * d * 2 * (frac_k + frac_v)
+    per_block_hbm = (1 - frac_v) * (BLOCK * d // 2 + BLOCK * (d // 32) * 8 + 4) + \
+        (1 - frac_k) * w.group * BLOCK * 4
+    units_per_launch = B * Hkv * nb_mid
+    att_h2d = per_block_h2d * units_per_launch
+    att_hbm = per_block_hbm * units_per_launch
+    t_h2d = att_h2d / (h2d_peak * 1e9)
+    t_hbm = att_hbm / (peaks["hbm_gbs"] * 1e9)
+    bound_h2d = t_h2d >= t_hbm
+    rec_att = traffic_record("attend")
+    roofline = {
+        "kernel": "attend (split-K attention, fused FP16 promotion from pinned Tier 2)",
+        "bound": "h2d" if bound_h2d else "hbm",
+        "achieved": (att_h2d if bound_h2d else att_hbm) / (att_ms * 1e-3) / 1e9,
+        "peak": h2d_peak if bound_h2d else peaks["hbm_gbs"],
+        "unit": "GB/s",
+        "peak_source": ("pinned cudaMemcpyAsync H2D probe, this run" if bound_h2d
+                        else f"MEASURED_PEAKS.json hbm_gbs ({peaks['source']})"),
+        "avg_launch_ms": att_ms,
+        "algorithmic_bytes_per_launch": {"host_link": att_h2d, "hbm": att_hbm},
+        "traffic": (rec_att["dram_bytes_per_block"] * units_per_launch if rec_att else None),
+    }
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+
+    sc_ms = phase_ms["score"] / max(1, phase_n["score"])
+    sc_bytes = units_per_launch * (BLOCK * d + 4 * d + w.group * BLOCK * 4 + 8 * w.group)
+    rec_sc = traffic_record("score")
+    roofline_hbm = {
+        "kernel": "score (INT8 scoring + block log-mass + Delta)",
+        "bound": "hbm", "achieved": sc_bytes / (sc_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peaks['source']}), of measured",
+        "avg_launch_ms": sc_ms, "algorithmic_bytes_per_launch": sc_bytes,
+        "traffic": (rec_sc["dram_bytes_per_block"] * units_per_launch if rec_sc else None),
+    }
+    roofline_hbm["frac"] = roofline_hbm["achieved"] / roofline_hbm["peak"]
+
+    nphase_ms, nphase_n, _ = nprof
+    quant_ms = sum(nphase_ms[p] for p in ("score", "select", "attend", "combine")) / n_naive
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "steps/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "layers": L, "global_batch": B * ws, "batch_per_gpu": B,
+            "ctx": w.ctx, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
+            "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
+            "l2": "inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (
+                t1_bytes / 2 ** 30),
+            "thresholds": dataclasses.asdict(th),
+        },
+        "roofline": roofline,
+        "roofline_hbm": roofline_hbm,
+        "int8_int4_path": {
+            "steps_per_s": n_naive * ws / n_max,
+            "effective_kv_gbs": kv_gbs,
+            "frac_of_hbm_peak": kv_gbs / ws / peaks["hbm_gbs"],
+            "tier1_bytes_per_step": t1_bytes,
+            "kernel_ms_per_step": quant_ms,
+            "kernel_kv_gbs": t1_bytes / (quant_ms * 1e-3) / 1e9,
+        },
+        "promotion": {
+            "key_promoted_frac": frac_k, "value_promoted_frac": frac_v,
+            "h2d_peak_gbs": h2d_peak,
+            "rung_histogram": census["rungs"],
+        },
+        "phases_ms_per_step": {k: v / n_steps for k, v in phase_ms.items()},
+        "gpu_launches": int(sum(phase_n.values())),
+        "clocks": clk,
+    }
+    if e2e:
+        res["e2e"] = e2e
+    cache.close()
+    return res
+
+
+# --------------------------------------------------------- oracle timing ----
+
+def oracle_sample_seconds(w: sk.Workload, layer: int, b: int, th) -> tuple[float, dict]:
+    """Time the CPU oracle's decode of one (layer, batch row) of the workload."""
+    from oracle import Thresholds as OT
+    from oracle import build_unit, decode
+    K, V = sk.kv_layer(w, layer, 0, w.ctx, device="cpu")
+    units = [build_unit(K[b, g].numpy(), V[b, g].numpy()) for g in range(w.n_kv_heads)]
+    q = sk.queries(w, layer, 0, "cpu")[b].numpy()
+    d = th.float32_rounded()
+    oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
+             rank_r=d["rank_r"], max_expand=d["max_expand"],
+             layer_dense_frac=d["layer_dense_frac"])
+    t0 = time.perf_counter()
+    decode(q, units, oth)
+    return time.perf_counter() - t0, units
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: sk.Workload, th, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands, on one (layer, batch row) at a time, scaled to steps/s."""
+    secs, n = [], 0
+    t_start = time.perf_counter()
+    layer = 0
+    while n < 1 or (time.perf_counter() - t_start < budget_s and n < 3):
+        s, _ = oracle_sample_seconds(w, layer % w.n_layers, 0, th)
+        secs.append(s)
+        n += 1
+        layer += 1
+    per = statistics.mean(secs)
+    step_s = per * w.n_layers * w.batch
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.n_layers * w.batch} (layer, batch row) decodes of one step, "
+                      f"{per:.2f} s each, scaled to the full step (appends not included)"}
+
+
+def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
+    import certified_quantized_kv_int8_b200 as cqa_py  # Thresholds only; no library call
+    if rank != 0:
+        return None
+    th = cqa_py.Thresholds(**sk.default_thresholds(w))
+    K, V = sk.kv_layer(w, 0, 0, w.ctx, device="cpu")
+    from oracle import Thresholds as OT
+    from oracle import build_unit, decode
+    units = [build_unit(K[0, g].numpy(), V[0, g].numpy()) for g in range(w.n_kv_heads)]
+    d = th.float32_rounded()
+    oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
+             rank_r=d["rank_r"], max_expand=d["max_expand"],
+             layer_dense_frac=d["layer_dense_frac"])
+    qs = [sk.queries(w, 0, s, "cpu")[0].numpy() for s in range(args.warmup + args.steps)]
+    for s in range(args.warmup):
+        decode(qs[s], units, oth)
+    t0 = time.perf_counter()
+    for s in range(args.warmup, args.warmup + args.steps):
+        decode(qs[s], units, oth)
+    el = time.perf_counter() - t0
+    per = el / args.steps
+    value = 1.0 / (per * w.n_layers * w.batch)
+    sample = (f"each step decodes one (layer 0, batch row 0) of the {w.n_layers}-layer, "
+              f"batch-{w.batch} step ({per:.2f} s) and is scaled by {w.n_layers * w.batch}")
+    return {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "steps/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per * w.n_layers * w.batch * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.n_layers, "global_batch": w.batch,
+                   "ctx": w.ctx, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(sk.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the nvidia-smi samples of the timed region in this file")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = sk.WORKLOADS[args.workload]
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        res = run_reference(args, w, ws, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    from certified_quantized_kv_int8_b200.build import build
+    if rank == 0:
+        build()
+    dist = init_dist(ws, "nccl")
+    if dist is not None:
+        barrier(dist, torch.device("cuda", local))
+        build()  # no-op once rank 0 built it
+    device = torch.device("cuda", local)
+    res = run_ours(args, w, ws, rank, dist, device)
+    if rank == 0 and res is not None:
+        if ws == 1 and not args.no_cpu_baseline:
+            import certified_quantized_kv_int8_b200 as cqa
+            res["cpu_baseline"] = cpu_baseline(w, cqa.Thresholds(**sk.default_thresholds(w)))
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,62 @@
+"""Host-side logic of bench.py: the max-over-ranks timing and the weak-scaling
+value, run as two gloo ranks on the CPU; and the reference (oracle) arm."""
+
+import json
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, ws, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(ws),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    dist = bench.init_dist(ws, "gloo", timeout_s=30)
+    dev = torch.device("cpu")
+    elapsed = 1.0 + rank  # rank 1 is the slowest
+    bench.barrier(dist, dev)
+    t = bench.max_over_ranks(elapsed, dist, dev)
+    v = bench.weak_scaling_value(10, ws, t)
+    with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+        json.dump({"t": t, "v": v}, f)
+    dist.destroy_process_group()
+
+
+def test_two_rank_timing_is_max_and_value_is_weak_scaling(tmp_path):
+    ws = 2
+    mp.start_processes(_rank_main, args=(ws, _free_port(), str(tmp_path)), nprocs=ws,
+                       join=True, start_method="spawn")
+    for r in range(ws):
+        d = json.load(open(tmp_path / f"r{r}.json"))
+        assert d["t"] == 2.0
+        assert d["v"] == pytest.approx(10 * 2 / 2.0)
+
+
+def test_single_process_helpers():
+    dev = torch.device("cpu")
+    assert bench.max_over_ranks(3.5, None, dev) == 3.5
+    assert bench.weak_scaling_value(20, 1, 2.0) == 10.0
+    assert bench.tier1_bytes_per_block(128) == 64 * 128 + 512 + 64 * 64 + 64 * 4 * 8 + 4
+
+
+def test_reference_arm_prints_one_line(capsys):
+    """--impl reference times the CPU oracle on a bounded sample (tiny workload)."""
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "3"])
+    assert rc == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
