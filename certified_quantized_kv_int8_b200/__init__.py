@@ -29,7 +29,7 @@ __all__ = [
     "CqaError", "Thresholds", "Cache", "load_library",
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
-    "cqa_profile_begin", "cqa_profile_end", "PHASES",
+    "cqa_profile_begin", "cqa_profile_end", "PHASES", "cqa_dense_attention_noalloc",
     "EXPORT_KCODES", "EXPORT_KSCALE", "EXPORT_VCODES", "EXPORT_VMETA", "EXPORT_ETA",
     "EXPORT_VRANGE", "EXPORT_RESIDUAL", "EXPORT_TIER2",
 ]
@@ -40,7 +40,7 @@ EXPORT_ETA, EXPORT_VRANGE, EXPORT_RESIDUAL, EXPORT_TIER2 = 4, 5, 6, 7
 EXPORTED_SYMBOLS = (
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
-    "cqa_profile_begin", "cqa_profile_end",
+    "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
 )
 
 PHASES = ("append_seal", "append_tail", "score", "select", "attend", "combine",
@@ -125,11 +125,12 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_profile_begin.argtypes = [vp, i32]
     lib.cqa_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int64)]
+    lib.cqa_dense_attention_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
                  "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
-                 "cqa_profile_begin", "cqa_profile_end"):
+                 "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -222,6 +223,22 @@ def cqa_profile_end(handle):
     untimed = _check(load_library().cqa_profile_end(handle, ms, n), "cqa_profile_end")
     return ({p: ms[i] for i, p in enumerate(PHASES)}, {p: int(n[i]) for i, p in enumerate(PHASES)},
             untimed)
+
+
+def cqa_dense_attention_noalloc(q, k, v, out, stream=None):
+    """Exact attention over caller-held FP16 keys and values that allocates no
+    device memory (for callers that cannot call cudaMalloc; see include/cqa.h).
+    q: CUDA float16 [batch][n_q_heads][head_dim]; k, v: CUDA float16
+    [batch][n_kv_heads][n_tokens][head_dim]; out: CUDA float32 like q."""
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = k.shape
+    _dev(q, torch.float16, (B, Hq, d), "q")
+    _dev(k, torch.float16, (B, Hkv, T, d), "k")
+    _dev(v, torch.float16, (B, Hkv, T, d), "v")
+    _dev(out, torch.float32, (B, Hq, d), "out")
+    return _check(load_library().cqa_dense_attention_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, d, T, _ptr(out), _stream(stream)),
+        "cqa_dense_attention_noalloc")
 
 
 class Cache:

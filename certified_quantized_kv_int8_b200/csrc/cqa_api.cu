@@ -125,7 +125,7 @@ const char* cqa_error_string(int code) {
     case CQA_ERR_INVALID_ARG: return "invalid argument";
     case CQA_ERR_CUDA: return "CUDA runtime error";
     case CQA_ERR_OOM: return "out of memory";
-    case CQA_ERR_CAPACITY: return "append exceeds the cache capacity (max_ctx)";
+    case CQA_ERR_CAPACITY: return "size exceeds a fixed capacity (cache max_ctx or scratch size)";
     case CQA_ERR_EMPTY: return "decode on an empty layer";
   }
   return "unknown error";

@@ -50,7 +50,7 @@ enum {
   CQA_ERR_INVALID_ARG = -1, /* null pointer, bad shape, layer out of range, ... */
   CQA_ERR_CUDA = -2,        /* a CUDA runtime call failed */
   CQA_ERR_OOM = -3,         /* device or pinned-host allocation failed */
-  CQA_ERR_CAPACITY = -4,    /* the append would exceed max_ctx */
+  CQA_ERR_CAPACITY = -4,    /* an append beyond max_ctx, or a shape beyond a fixed scratch size */
   CQA_ERR_EMPTY = -5        /* decode on a layer that holds no token */
 };
 
@@ -192,6 +192,39 @@ int cqa_profile_begin(cqa_cache* cache, int max_launches);
  * arrays (either may be NULL).  Returns the number of launches left untimed
  * (>= 0) or a negative error. */
 int cqa_profile_end(cqa_cache* cache, double* ms, int64_t* launches);
+
+/* Size in bytes of the fixed device scratch array that
+ * cqa_dense_attention_noalloc uses (every device that loads the library holds
+ * one such array until the process exits). */
+#define CQA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* Exact attention softmax(q K^T / sqrt(head_dim)) V over FP16 keys and values
+ * that the caller holds in device memory, computed without allocating any
+ * memory.  The paper has no counterpart of this entry point: it exists for
+ * callers that cannot call cudaMalloc, e.g. code running while a stream is
+ * captured into a CUDA graph (an allocation there fails or breaks the
+ * capture), hosts whose single allocator is owned by another framework under
+ * a fixed memory budget, and latency-critical paths where cudaMalloc/cudaFree
+ * may synchronise the device.
+ *
+ * q_fp16: device fp16 [batch][n_q_heads][head_dim]; k_fp16, v_fp16: device
+ * fp16 [batch][n_kv_heads][n_tokens][head_dim]; out: device fp32
+ * [batch][n_q_heads][head_dim]; all 16-byte aligned, owned by the caller.
+ * The split-K partials live in a file-scope device array of
+ * CQA_NOALLOC_SCRATCH_BYTES; shapes whose partials cannot fit (batch *
+ * n_kv_heads * (n_q_heads / n_kv_heads) * (head_dim + 3) * 4 bytes above it)
+ * are rejected with CQA_ERR_CAPACITY before anything is launched.  The call
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on a device (the current device) looks up the array's device
+ * address with cudaGetSymbolAddress; make that first call before any stream
+ * capture.  Every call on a device shares the one array, which keeps the last
+ * call's contents (each call rewrites every partial before reading it, so
+ * nothing needs clearing); calls that overlap on the GPU race on it, so
+ * serialise them (one stream, or streams ordered by events). */
+int cqa_dense_attention_noalloc(const void* q_fp16, const void* k_fp16, const void* v_fp16,
+                                int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                int n_tokens, float* out, void* stream);
 
 /* Static description of an error code. */
 const char* cqa_error_string(int code);

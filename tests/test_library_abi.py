@@ -45,6 +45,7 @@ def test_library_loads_and_binding_matches(libpath):
     assert set(cqa.EXPORTED_SYMBOLS) == set(_declared_entry_points())
     assert cqa.cqa_error_string(0) == "ok"
     assert "capacity" in cqa.cqa_error_string(-4)
+    assert cqa.cqa_error_string(12345) == "unknown error"
 
 
 def test_binding_reports_a_missing_library(tmp_path, monkeypatch):
