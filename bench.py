@@ -197,6 +197,64 @@ def traffic_record(kernel: str):
     return rec
 
 
+def decision_census(cache, qs, th, w, device) -> dict:
+    """Decode every layer once more with a trace and count the decisions."""
+    L, B, Hkv, G = w.n_layers, w.batch, w.n_kv_heads, w.group
+    c = dict(blocks=0, key_promoted=0, value_promoted=0, heads=0, rungs=[0] * 5, units=0,
+             dense_units=0, dense_unit_blocks=0, dense_unit_nonpromoted=0,
+             vp_or_dense_blocks=0, int4_blocks=0, blocks_per_layer=0)
+    for layer in range(L):
+        tr = cache.alloc_trace(layer)
+        o = cache.alloc_outputs()
+        cache.decode(layer, qs[layer], th, outputs=o, trace=tr)
+        torch.cuda.synchronize(device)
+        nb = cache.length(layer) // BLOCK
+        bf = tr["block_flags"].cpu().numpy()[..., :nb]  # [B][Hkv][nb]
+        rg = o[3].cpu().numpy()  # [B][Hq]
+        dense_h = rg.reshape(B, Hkv, G) >= 3
+        unit_dense = dense_h.any(axis=2)  # [B][Hkv]
+        unit_mixed = (~dense_h).any(axis=2)
+        kp = (bf & 1).astype(bool)
+        vp = (bf & 2).astype(bool)
+        c["blocks"] += int(bf.size)
+        c["blocks_per_layer"] = B * Hkv * nb
+        c["key_promoted"] += int(kp.sum())
+        c["value_promoted"] += int(vp.sum())
+        c["units"] += B * Hkv
+        c["dense_units"] += int(unit_dense.sum())
+        c["dense_unit_blocks"] += int(unit_dense.sum()) * nb
+        c["dense_unit_nonpromoted"] += int((~kp & unit_dense[..., None]).sum())
+        c["vp_or_dense_blocks"] += int((vp | unit_dense[..., None]).sum())
+        c["int4_blocks"] += int((~vp & unit_mixed[..., None]).sum())
+        c["heads"] += int(rg.size)
+        for r in range(5):
+            c["rungs"][r] += int((rg == r).sum())
+    return c
+
+
+def phase_bytes(c: dict, w: sk.Workload, staged_frac: float = 0.0) -> dict:
+    """Algorithmic bytes per launch of each decode phase: (host link, HBM).
+    staged_frac: share of promote launches whose keys came from the device copy
+    made by the whole-layer key prefetch (read from HBM instead of Tier 2)."""
+    L, d, G = w.n_layers, w.head_dim, w.group
+    kblk = BLOCK * d * 2  # FP16 keys (or values) of one block and kv head
+    per = lambda x: x / L  # noqa: E731  (census counts are over all layers)
+    nblk = per(c["blocks"])
+    kp = per(c["key_promoted"]) * kblk
+    return {
+        "score": (0.0, nblk * (BLOCK * d + 4 * d + G * BLOCK * 4 + 8 * G)),
+        "select": (0.0, nblk * (G * 12 + 5)),
+        "promote": ((1 - staged_frac) * kp,
+                    staged_frac * kp + per(c["key_promoted"]) * G * (BLOCK * 4 + 4)),
+        "prefetch": (nblk * kblk, nblk * kblk),
+        "dense_keys": (per(c["dense_unit_nonpromoted"]) * kblk,
+                       per(c["dense_unit_nonpromoted"]) * G * BLOCK * 4),
+        "attend": (per(c["vp_or_dense_blocks"]) * kblk,
+                   per(c["int4_blocks"]) * (BLOCK * d // 2 + BLOCK * (d // 32) * 8 + 4)
+                   + nblk * G * BLOCK * 4),
+    }
+
+
 # --------------------------------------------------------------- our arm ----
 
 def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | None:
@@ -268,24 +326,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     phase_ms, phase_n, untimed = prof
 
     # census of the decisions (untimed, on the state after the timed steps)
-    census = dict(blocks=0, key_promoted=0, value_promoted=0, heads=0,
-                  rungs=[0, 0, 0, 0, 0])
-    for layer in range(L):
-        tr = cache.alloc_trace(layer)
-        o = cache.alloc_outputs()
-        cache.decode(layer, inputs[args.warmup + args.steps - 1][0][layer], th, outputs=o,
-                     trace=tr)
-        torch.cuda.synchronize(device)
-        bf = tr["block_flags"].cpu().numpy()
-        nb = cache.length(layer) // BLOCK
-        bf = bf[..., :nb]
-        census["blocks"] += int(bf.size)
-        census["key_promoted"] += int((bf & 1).astype(bool).sum())
-        census["value_promoted"] += int((bf & 2).astype(bool).sum())
-        rg = o[3].cpu().numpy().ravel()
-        census["heads"] += int(rg.size)
-        for r in range(5):
-            census["rungs"][r] += int((rg == r).sum())
+    census = decision_census(cache, inputs[args.warmup + args.steps - 1][0], th, w, device)
 
     # end to end through the public API: host inputs in, host results out, every step
     e2e = None
@@ -333,51 +374,54 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
 
     h2d_peak = h2d_probe_gbs(device)
 
-    # dominant kernel of the certified step
-    n_steps = args.steps
-    att_ms = phase_ms["attend"] / max(1, phase_n["attend"])
-    ctx_mid = cache.length(0)
-    nb_mid = ctx_mid // BLOCK
-    frac_k = census["key_promoted"] / max(1, census["blocks"])
-    frac_v = census["value_promoted"] / max(1, census["blocks"])
-    per_block_h2d = BLOCK * d * 2 * (frac_k + frac_v)
-    per_block_hbm = (1 - frac_v) * (BLOCK * d // 2 + BLOCK * (d // 32) * 8 + 4) + \
-        (1 - frac_k) * w.group * BLOCK * 4
-    units_per_launch = B * Hkv * nb_mid
-    att_h2d = per_block_h2d * units_per_launch
-    att_hbm = per_block_hbm * units_per_launch
-    t_h2d = att_h2d / (h2d_peak * 1e9)
-    t_hbm = att_hbm / (peaks["hbm_gbs"] * 1e9)
-    bound_h2d = t_h2d >= t_hbm
-    rec_att = traffic_record("attend")
+    # per-phase algorithmic bytes per launch, from the decisions of the census
+    staged = phase_n["prefetch"] / max(1, phase_n["promote"])
+    pb = phase_bytes(census, w, staged_frac=min(1.0, staged))
+    phases = {}
+    for p_, ms in phase_ms.items():
+        n = phase_n[p_]
+        if n == 0 or p_ not in pb:
+            continue
+        host_b, hbm_b = pb[p_]
+        avg = ms / n
+        t_host = host_b / (h2d_peak * 1e9)
+        t_hbm = hbm_b / (peaks["hbm_gbs"] * 1e9)
+        bound = "h2d" if t_host >= t_hbm else "hbm"
+        ach = (host_b if bound == "h2d" else hbm_b) / (avg * 1e-3) / 1e9
+        pk = h2d_peak if bound == "h2d" else peaks["hbm_gbs"]
+        phases[p_] = {"ms_per_step": ms / args.steps, "launches": n, "avg_launch_ms": avg,
+                      "host_link_bytes": host_b, "hbm_bytes": hbm_b, "bound": bound,
+                      "achieved_gbs": ach, "frac": ach / pk}
+    # the dominant kernel (the prefetch is a copy-engine transfer, not a kernel)
+    dom = max((k for k in phases if k != "prefetch"), key=lambda k: phases[k]["ms_per_step"])
+    dp = phases[dom]
+    rec = traffic_record(dom)
     roofline = {
-        "kernel": "attend (split-K attention, fused FP16 promotion from pinned Tier 2)",
-        "bound": "h2d" if bound_h2d else "hbm",
-        "achieved": (att_h2d if bound_h2d else att_hbm) / (att_ms * 1e-3) / 1e9,
-        "peak": h2d_peak if bound_h2d else peaks["hbm_gbs"],
-        "unit": "GB/s",
-        "peak_source": ("pinned cudaMemcpyAsync H2D probe, this run" if bound_h2d
-                        else f"MEASURED_PEAKS.json hbm_gbs ({peaks['source']})"),
-        "avg_launch_ms": att_ms,
-        "algorithmic_bytes_per_launch": {"host_link": att_h2d, "hbm": att_hbm},
-        "traffic": (rec_att["dram_bytes_per_block"] * units_per_launch if rec_att else None),
+        "kernel": dom, "bound": dp["bound"], "achieved": dp["achieved_gbs"],
+        "peak": h2d_peak if dp["bound"] == "h2d" else peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": dp["frac"],
+        "peak_source": ("pinned 1 GiB cudaMemcpyAsync H2D probe, this run" if dp["bound"] == "h2d"
+                        else f"MEASURED_PEAKS.json hbm_gbs, of {peaks['source']}"),
+        "avg_launch_ms": dp["avg_launch_ms"],
+        "algorithmic_bytes_per_launch": {"host_link": dp["host_link_bytes"],
+                                         "hbm": dp["hbm_bytes"]},
+        "traffic": (rec["dram_bytes_per_block"] * census["blocks_per_layer"] if rec else None),
     }
-    roofline["frac"] = roofline["achieved"] / roofline["peak"]
-
-    sc_ms = phase_ms["score"] / max(1, phase_n["score"])
-    sc_bytes = units_per_launch * (BLOCK * d + 4 * d + w.group * BLOCK * 4 + 8 * w.group)
+    sp = phases["score"]
     rec_sc = traffic_record("score")
     roofline_hbm = {
-        "kernel": "score (INT8 scoring + block log-mass + Delta)",
-        "bound": "hbm", "achieved": sc_bytes / (sc_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
-        "unit": "GB/s", "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peaks['source']}), of measured",
-        "avg_launch_ms": sc_ms, "algorithmic_bytes_per_launch": sc_bytes,
-        "traffic": (rec_sc["dram_bytes_per_block"] * units_per_launch if rec_sc else None),
+        "kernel": "score", "bound": "hbm", "achieved": sp["hbm_bytes"] / (sp["avg_launch_ms"] * 1e-3) / 1e9,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "peak_source": f"MEASURED_PEAKS.json hbm_gbs, of {peaks['source']}",
+        "avg_launch_ms": sp["avg_launch_ms"], "algorithmic_bytes_per_launch": sp["hbm_bytes"],
+        "traffic": (rec_sc["dram_bytes_per_block"] * census["blocks_per_layer"] if rec_sc else None),
     }
     roofline_hbm["frac"] = roofline_hbm["achieved"] / roofline_hbm["peak"]
+    frac_k = census["key_promoted"] / max(1, census["blocks"])
+    frac_v = census["value_promoted"] / max(1, census["blocks"])
 
     nphase_ms, nphase_n, _ = nprof
-    quant_ms = sum(nphase_ms[p] for p in ("score", "select", "attend", "combine")) / n_naive
+    quant_ms = sum(v for k, v in nphase_ms.items() if not k.startswith("append")) / n_naive
     res = {
         "metric": METRIC,
         "value": value,
@@ -411,11 +455,14 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         },
         "promotion": {
             "key_promoted_frac": frac_k, "value_promoted_frac": frac_v,
+            "dense_unit_frac": census["dense_units"] / max(1, census["units"]),
             "h2d_peak_gbs": h2d_peak,
+            "staged_layer_frac": staged,
+            "prefetch_copy_gbs": phases.get("prefetch", {}).get("achieved_gbs"),
             "rung_histogram": census["rungs"],
         },
-        "phases_ms_per_step": {k: v / n_steps for k, v in phase_ms.items()},
-        "gpu_launches": int(sum(phase_n.values())),
+        "phases": phases,
+        "gpu_launches": int(sum(v for k, v in phase_n.items() if k != "prefetch")),
         "clocks": clk,
     }
     if e2e:

@@ -30,6 +30,7 @@ __all__ = [
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "PHASES", "cqa_dense_attention_noalloc",
+    "cqa_set_key_prefetch",
     "EXPORT_KCODES", "EXPORT_KSCALE", "EXPORT_VCODES", "EXPORT_VMETA", "EXPORT_ETA",
     "EXPORT_VRANGE", "EXPORT_RESIDUAL", "EXPORT_TIER2",
 ]
@@ -41,10 +42,11 @@ EXPORTED_SYMBOLS = (
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
+    "cqa_set_key_prefetch",
 )
 
-PHASES = ("append_seal", "append_tail", "score", "select", "attend", "combine",
-          "dense_attend", "dense_combine")
+PHASES = ("append_seal", "append_tail", "score", "select", "promote", "decide", "dense_keys",
+          "attend", "combine", "dense_attend", "dense_combine", "prefetch")
 
 
 class _Config(ctypes.Structure):
@@ -126,11 +128,13 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_profile_end.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.cqa_dense_attention_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    lib.cqa_set_key_prefetch.argtypes = [vp, i32, ctypes.c_float]
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
                  "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
-                 "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc"):
+                 "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
+                 "cqa_set_key_prefetch"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -225,6 +229,12 @@ def cqa_profile_end(handle):
             untimed)
 
 
+def cqa_set_key_prefetch(handle, mode: int = 1, min_fraction: float = 0.75):
+    """0 off, 1 adaptive (default), 2 always; see include/cqa.h."""
+    return _check(load_library().cqa_set_key_prefetch(handle, int(mode), float(min_fraction)),
+                  "cqa_set_key_prefetch")
+
+
 def cqa_dense_attention_noalloc(q, k, v, out, stream=None):
     """Exact attention over caller-held FP16 keys and values that allocates no
     device memory (for callers that cannot call cudaMalloc; see include/cqa.h).
@@ -267,6 +277,9 @@ class Cache:
 
     def __exit__(self, *exc):
         self.close()
+
+    def set_key_prefetch(self, mode: int = 1, min_fraction: float = 0.75):
+        return cqa_set_key_prefetch(self.handle, mode, min_fraction)
 
     def profile_begin(self, max_launches: int = 1 << 16):
         return cqa_profile_begin(self.handle, max_launches)

@@ -33,6 +33,16 @@ struct cqa_cache {
   size_t prof_max;
   int64_t prof_launches[CQA_PHASE_COUNT];
   int64_t prof_untimed;
+  // whole-layer key prefetch by the copy engine (cqa_set_key_prefetch)
+  int pref_mode;       // 0 off, 1 adaptive, 2 always
+  float pref_min_frac; // adaptive: the layer's last decode promoted at least this fraction
+  cudaStream_t side;   // copy stream
+  __half* kstage[2];   // [B*Hkv][max_ctx][d] device copies of one layer's Tier-2 keys
+  int stage_layer[2];  // layer held by each slot, -1 none
+  int stage_nb[2];     // sealed blocks copied into the slot
+  cudaEvent_t ev_ready[2], ev_free[2], ev_main;
+  int32_t* promo_host; // [n_layers * B * Hkv] promoted blocks of the last decode (mapped)
+  int32_t* promo_dev;
 };
 
 namespace {
@@ -113,6 +123,62 @@ cudaError_t run_phase(cqa_cache* c, int phase, cudaStream_t s, int nlaunch, F&& 
   }
   c->prof_launches[phase] += nlaunch;
   return e;
+}
+
+// Fraction of the layer's sealed blocks its last decode promoted (-1 unknown).
+double last_promoted_fraction(const cqa_cache* c, int layer, int nb) {
+  const size_t units = (size_t)c->cfg.batch * c->cfg.n_kv_heads;
+  const volatile int32_t* p = c->promo_host + (size_t)layer * units;
+  long long n = 0;
+  for (size_t i = 0; i < units; ++i) {
+    const int32_t v = p[i];
+    if (v < 0) return -1.0;
+    n += v;
+  }
+  return nb > 0 ? (double)n / ((double)units * nb) : -1.0;
+}
+
+bool want_prefetch(const cqa_cache* c, int layer) {
+  if (c->pref_mode == 0) return false;
+  const int nb = c->len[layer] / BLK;
+  if (nb == 0) return false;
+  if (c->pref_mode == 2) return true;
+  return last_promoted_fraction(c, layer, nb) >= c->pref_min_frac;
+}
+
+int staged_slot(const cqa_cache* c, int layer) {
+  for (int i = 0; i < 2; ++i)
+    if (c->stage_layer[i] == layer) return i;
+  return -1;
+}
+
+// Copy the sealed blocks of `layer`'s Tier-2 keys into a device slot on the
+// copy stream, after all work already queued on `s` (the appends that wrote
+// them) and after the slot's last reader.  Returns the slot or -1.
+int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
+  const int nb = c->len[layer] / BLK;
+  if (nb == 0) return -1;
+  int slot = staged_slot(c, layer);
+  if (slot >= 0 && c->stage_nb[slot] == nb) return slot;
+  if (slot < 0) slot = (avoid_slot == 0) ? 1 : 0;
+  const size_t units = (size_t)c->cfg.batch * c->cfg.n_kv_heads;
+  const size_t pitch = c->st.tier2 * 2;
+  const char* src = (const char*)c->k2_host + (size_t)layer * units * pitch;
+  if (cudaEventRecord(c->ev_main, s) != cudaSuccess) return -1;
+  if (cudaStreamWaitEvent(c->side, c->ev_main, 0) != cudaSuccess) return -1;
+  if (cudaStreamWaitEvent(c->side, c->ev_free[slot], 0) != cudaSuccess) return -1;
+  const int timed = c->prof_on ? 1 : 0;
+  cudaError_t e = run_phase(c, CQA_PHASE_PREFETCH, c->side, timed, [&] {
+    return cudaMemcpy2DAsync(c->kstage[slot], pitch, src, pitch, (size_t)nb * BLK * c->cfg.head_dim * 2,
+                             units, cudaMemcpyHostToDevice, c->side);
+  });
+  if (e != cudaSuccess || cudaEventRecord(c->ev_ready[slot], c->side) != cudaSuccess) {
+    c->stage_layer[slot] = -1;
+    return -1;
+  }
+  c->stage_layer[slot] = layer;
+  c->stage_nb[slot] = nb;
+  return slot;
 }
 
 }  // namespace
@@ -260,6 +326,39 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
     cqa_cache_destroy(cc);
     return CQA_ERR_OOM;
   }
+  // key prefetch: two device slots of one layer's keys, a copy stream, events
+  cc->pref_mode = 1;
+  cc->pref_min_frac = 0.75f;
+  cc->stage_layer[0] = cc->stage_layer[1] = -1;
+  const size_t layer_units = (size_t)c.batch * c.n_kv_heads;
+  const size_t stage_bytes = layer_units * st.tier2 * 2;
+  if (cudaMalloc(&cc->kstage[0], stage_bytes) != cudaSuccess ||
+      cudaMalloc(&cc->kstage[1], stage_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    cqa_cache_destroy(cc);
+    return CQA_ERR_OOM;
+  }
+  if (cudaStreamCreateWithFlags(&cc->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&cc->ev_ready[0], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&cc->ev_ready[1], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&cc->ev_free[0], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&cc->ev_free[1], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&cc->ev_main, cudaEventDisableTiming) != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+  if (cudaHostAlloc((void**)&cc->promo_host, units * sizeof(int32_t),
+                    cudaHostAllocMapped | cudaHostAllocPortable) != cudaSuccess) {
+    cudaGetLastError();
+    cqa_cache_destroy(cc);
+    return CQA_ERR_OOM;
+  }
+  memset(cc->promo_host, 0xff, units * sizeof(int32_t));  // -1: no decode yet
+  if (cudaHostGetDevicePointer((void**)&cc->promo_dev, cc->promo_host, 0) != cudaSuccess) {
+    cqa_cache_destroy(cc);
+    return CQA_ERR_CUDA;
+  }
+  cc->sc.promo = cc->promo_dev;
   if (cudaDeviceSynchronize() != cudaSuccess) {
     cqa_cache_destroy(cc);
     return CQA_ERR_CUDA;
@@ -279,6 +378,14 @@ int cqa_cache_destroy(cqa_cache* cc) {
     if (cc->v2_host) cudaFreeHost(cc->v2_host);
     if (cc->prof_events)
       for (cudaEvent_t ev : *cc->prof_events) cudaEventDestroy(ev);
+    for (int i = 0; i < 2; ++i) {
+      if (cc->kstage[i]) cudaFree(cc->kstage[i]);
+      if (cc->ev_ready[i]) cudaEventDestroy(cc->ev_ready[i]);
+      if (cc->ev_free[i]) cudaEventDestroy(cc->ev_free[i]);
+    }
+    if (cc->ev_main) cudaEventDestroy(cc->ev_main);
+    if (cc->side) cudaStreamDestroy(cc->side);
+    if (cc->promo_host) cudaFreeHost(cc->promo_host);
   }
   delete cc->prof_events;
   delete cc->prof_phase;
@@ -362,19 +469,45 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   if (need < 0) need = 0;
   const int need_dense = need > 1e9 ? 1000000000 : (int)need;
   const __half* qh = (const __half*)q;
+  const bool naive = tv.naive != 0;
+  const bool post_check = !naive && !isinf(tv.eps_val);
+  // keys of this layer staged by an earlier call, or staged now; then the next layer's
+  int slot = -1;
+  if (!naive) {
+    slot = staged_slot(cc, layer);
+    if (slot >= 0 && cc->stage_nb[slot] != sh.nb) slot = -1;
+    if (slot < 0 && want_prefetch(cc, layer)) slot = issue_prefetch(cc, layer, -1, s);
+    const int next = (layer + 1) % cc->cfg.n_layers;
+    if (next != layer && want_prefetch(cc, next)) issue_prefetch(cc, next, slot, s);
+  }
+  const __half* kstage = slot >= 0 ? cc->kstage[slot] : nullptr;
+  const int stage_nb = slot >= 0 ? cc->stage_nb[slot] : 0;
   cudaError_t e = run_phase(cc, CQA_PHASE_SCORE, s, 1,
                             [&] { return launch_score(cc->t, cc->st, unit0, sh, qh, cc->sc, s); });
   if (e == cudaSuccess)
     e = run_phase(cc, CQA_PHASE_SELECT, s, 1,
                   [&] { return launch_select(cc->t, cc->st, unit0, sh, tv, cc->sc, s); });
+  if (e == cudaSuccess && slot >= 0) e = cudaStreamWaitEvent(s, cc->ev_ready[slot], 0);
+  if (e == cudaSuccess && !naive && sh.nb > 0)
+    e = run_phase(cc, CQA_PHASE_PROMOTE, s, 1, [&] {
+      return launch_promote(cc->t, cc->st, unit0, sh, qh, cc->sc, 0, kstage, stage_nb, s);
+    });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_DECIDE, s, 1,
+                  [&] { return launch_decide(sh, tv, need_dense, cc->sc, s); });
+  if (e == cudaSuccess && !naive && sh.nb > 0)
+    e = run_phase(cc, CQA_PHASE_DENSE_KEYS, s, 1, [&] {
+      return launch_promote(cc->t, cc->st, unit0, sh, qh, cc->sc, 1, kstage, stage_nb, s);
+    });
+  if (e == cudaSuccess && slot >= 0) e = cudaEventRecord(cc->ev_free[slot], s);
   if (e == cudaSuccess)
     e = run_phase(cc, CQA_PHASE_ATTEND, s, 1,
                   [&] { return launch_attend(cc->t, cc->st, unit0, sh, qh, cc->sc, 0, s); });
   if (e == cudaSuccess)
     e = run_phase(cc, CQA_PHASE_COMBINE, s, 1, [&] {
-      return launch_combine(sh, tv, need_dense, cc->sc, out, e_key, e_val, rung, s);
+      return launch_combine(sh, tv, cc->sc, out, e_key, e_val, rung, s);
     });
-  if (e == cudaSuccess && !tv.naive) {
+  if (e == cudaSuccess && post_check) {
     e = run_phase(cc, CQA_PHASE_DENSE_ATTEND, s, 1,
                   [&] { return launch_attend(cc->t, cc->st, unit0, sh, qh, cc->sc, 1, s); });
     if (e == cudaSuccess)
@@ -456,6 +589,14 @@ int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t b
     }
   }
   return (int64_t)total;
+}
+
+int cqa_set_key_prefetch(cqa_cache* cc, int mode, float min_fraction) {
+  if (!cc || mode < 0 || mode > 2 || !(min_fraction >= 0.f && min_fraction <= 1.f))
+    return CQA_ERR_INVALID_ARG;
+  cc->pref_mode = mode;
+  cc->pref_min_frac = min_fraction;
+  return CQA_OK;
 }
 
 int cqa_profile_begin(cqa_cache* cc, int max_launches) {

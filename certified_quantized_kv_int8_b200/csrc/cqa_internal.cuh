@@ -32,6 +32,10 @@ constexpr uint8_t HF_VALUE = 2;
 constexpr uint8_t HF_KEYFAIL = 4;
 constexpr uint8_t HF_RANKFAIL = 8;
 constexpr uint8_t HF_VALFAIL = 16;
+// dense-flag byte: 3 or 4 = rung decided before the attention pass (its exact
+// logits and FP16 values are used there); DENSE_LATE marks an E_val post-check
+// failure that a separate dense pass recomputes
+constexpr uint8_t DENSE_LATE = 0x80;
 
 struct Tier1 {
   int8_t* kcodes;
@@ -78,6 +82,7 @@ struct Scratch {
   uint8_t* dense;    // [B][Hq] 0, 3 or 4
   float* part_o;     // [B*Hkv][max_chunks][G][d]
   float* part_s;     // [B*Hkv][max_chunks][G][3]  (m, l, eta mass)
+  int32_t* promo;    // [n_layers * B * Hkv] promoted block count per unit (pinned host, mapped)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
 };
@@ -96,16 +101,26 @@ cudaError_t launch_append_tail(const Tier1& t, const Strides& st, int layer_unit
                                int n_new, int nb_new, cudaStream_t s);
 cudaError_t launch_score(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
                          const __half* q, const Scratch& sc, cudaStream_t s);
+// mode 0: promoted blocks (exact logits in place, ell16); 1: the other blocks
+// of units holding a dense head (exact logits of the dense heads).  Keys of
+// blocks j < stage_nb are read from `kstage` (a device copy of the layer's
+// Tier-2 keys, same per-unit layout), the others from Tier 2.
+cudaError_t launch_promote(const Tier1& t, const Strides& st, int layer_unit0,
+                           const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
+                           const __half* kstage, int stage_nb, cudaStream_t s);
+cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
+                          const Scratch& sc, cudaStream_t s);
 cudaError_t launch_select(const Tier1& t, const Strides& st, int layer_unit0,
                           const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                           cudaStream_t s);
-// mode 0: certified (block flags decide), 1: dense for flagged heads, 2: dense for all
+// mode 0: certified (logits from scratch; block and dense flags choose the
+// values), 1: dense from Tier 2 for heads flagged DENSE_LATE, 2: dense for all
 cudaError_t launch_attend(const Tier1& t, const Strides& st, int layer_unit0,
                           const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
                           cudaStream_t s);
-cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
-                           const Scratch& sc, float* out, float* e_key, float* e_val,
-                           uint8_t* rung, cudaStream_t s);
+cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
+                           float* out, float* e_key, float* e_val, uint8_t* rung,
+                           cudaStream_t s);
 cudaError_t launch_dense_combine(const DecodeShape& sh, const Scratch& sc, int all_heads,
                                  float* out, float* e_key, float* e_val, uint8_t* rung,
                                  cudaStream_t s);

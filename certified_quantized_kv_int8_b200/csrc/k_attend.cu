@@ -1,5 +1,6 @@
 // Split-K decode attention over the tiered cache with the fused value-bound
-// accumulation, and the exact dense path used by rungs 3-4 and by
+// accumulation (the softmax and P.V pass of a certified decode step), and the
+// exact dense attention from Tier 2 used by the E_val post-check and by
 // cqa_dense_reference.
 //
 // Runtime-Certified Bounded-Error Quantized Attention, Methodology §1
@@ -9,10 +10,13 @@
 // keys, tail blocks keep their INT8 scores; the FP16 block log-masses of the
 // promoted blocks feed the rank-consistency check).
 //
-// Promotion is fused into this kernel: a promoted block's FP16 keys (and, for
-// value-promoted blocks, FP16 values) are read straight from the pinned,
-// device-mapped Tier 2 over the host link while other CTAs stream Tier-1 data
-// from HBM, so paging overlaps the tail work without a staging copy.
+// In a certified step the logits are already final when this pass runs: the
+// scoring pass wrote INT8 logits, the promotion pass replaced those of the
+// promoted blocks (and, for heads that fall back to dense attention, of every
+// block) with exact ones.  This pass reads them, chooses each block's values
+// per head (FP16 straight from the pinned, device-mapped Tier 2 for
+// value-promoted blocks and dense heads, INT4 from Tier 1 otherwise) and
+// accumulates the attention mass of INT4-valued blocks times eta_b.
 //
 // One CTA = (kv head unit, chunk of consecutive blocks), all G query heads;
 // chunk 0 also takes the exact residual block.  Per head the CTA keeps an
@@ -66,8 +70,13 @@ struct AttendSmem {
   float m[G], l[G], e[G], alpha[G];
 };
 
-// MODE 0: certified (block flags decide); 1: dense, only units holding a
-// flagged head; 2: dense for every head.
+// MODE 0: certified.  Logits come from scratch: INT8 for tail blocks, exact
+//         for promoted blocks, the residual, and every block of a dense head.
+//         Values per (block, head): FP16 from Tier 2 for value-promoted blocks
+//         and dense heads, INT4 from Tier 1 otherwise.
+// MODE 1: exact attention from Tier 2 keys and values for units holding a head
+//         flagged DENSE_LATE (the E_val post-check).
+// MODE 2: exact attention from Tier 2 for every head (cqa_dense_reference).
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, int unit0,
                                                          DecodeShape sh,
@@ -88,22 +97,35 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
   const int j0 = chunk * sh.chunk_blocks;
   const int j1 = min(sh.nb, j0 + sh.chunk_blocks);
 
+  // per head: exact (dense) or certified mixed attention
+  bool dh[G];
+  bool any_dense = false, any_mixed = false;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint8_t dv = sc.dense[hrow0 + h];
+    dh[h] = MODE == 0 ? (dv != 0) : true;
+    any_dense |= dh[h];
+    any_mixed |= !dh[h];
+  }
   if (MODE == 1) {
-    bool any = false;
-    for (int h = 0; h < G; ++h) any |= sc.dense[hrow0 + h] != 0;
-    if (!any) return;
+    bool late = false;
+#pragma unroll
+    for (int h = 0; h < G; ++h) late |= (sc.dense[hrow0 + h] & DENSE_LATE) != 0;
+    if (!late) return;
   }
 
   const int row = tid / LPR, cl = tid - row * LPR;  // row in pass, channel slice cl*8..cl*8+7
   float2 qr[G][4];
+  if (MODE != 0) {
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint4 qv = *reinterpret_cast<const uint4*>(q + (hrow0 + h) * D + cl * 8);
-    const __half2* qh = reinterpret_cast<const __half2*>(&qv);
+    for (int h = 0; h < G; ++h) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(q + (hrow0 + h) * D + cl * 8);
+      const __half2* qh = reinterpret_cast<const __half2*>(&qv);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __half22float2(qh[k]);
-      qr[h][k] = make_float2(f.x * sh.sigma, f.y * sh.sigma);
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(qh[k]);
+        qr[h][k] = make_float2(f.x * sh.sigma, f.y * sh.sigma);
+      }
     }
   }
   float2 acc[G][4];
@@ -125,13 +147,18 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
   for (int j = jstart; j < j1; ++j) {
     const bool resid = j < 0;
     const uint8_t fl = (MODE == 0 && !resid) ? bf[j] : (uint8_t)(BF_KEY | BF_VAL);
-    const bool kprom = resid || (fl & BF_KEY);  // residual: exact keys held on the device
     const bool vprom = resid || (fl & BF_VAL);
     const int ntok = resid ? sh.r : BLK;
-    const size_t tok0 = resid ? 0 : (size_t)j * BLK;
+    const size_t tok0 = resid ? (size_t)sh.nb * BLK : (size_t)j * BLK;  // token index
 
     // ---- logits ----
-    if (kprom) {
+    if (MODE == 0) {
+      const float* lp = sc.logits + hrow0 * sc.ls + tok0;
+      for (int e = tid; e < G * BLK; e += THREADS) {
+        const int h = e / BLK, tt = e - h * BLK;
+        S.lg[h][tt] = tt < ntok ? lp[h * sc.ls + tt] : -INFINITY;
+      }
+    } else {
       const __half* kb = resid ? t.kres + u * st.res : t.k2 + u * st.tier2 + tok0 * D;
       uint4 kv[NPASS];
 #pragma unroll
@@ -159,12 +186,6 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         for (int k = 0; k < LPR; ++k) s += S.u.kpart[h][tt][k];
         S.lg[h][tt] = tt < ntok ? s : -INFINITY;
       }
-    } else {
-      const float* lp = sc.logits + hrow0 * sc.ls + tok0;
-      for (int e = tid; e < G * BLK; e += THREADS) {
-        const int h = e / BLK, tt = e - h * BLK;
-        S.lg[h][tt] = lp[h * sc.ls + tt];
-      }
     }
     __syncthreads();
 
@@ -185,11 +206,11 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         const float lb = sb * c;
         S.l[h] = S.l[h] * alpha + lb;
         float ea = S.e[h] * alpha;
-        if (MODE == 0 && !vprom) ea += t.eta[u * st.eta + j] * lb;
+        const bool int4_here = MODE == 0 && !vprom && !sc.dense[hrow0 + h];
+        if (int4_here) ea += t.eta[u * st.eta + j] * lb;
         S.e[h] = ea;
         S.m[h] = mnew;
         S.alpha[h] = alpha;
-        if (MODE == 0 && !resid && kprom) sc.ell16[(hrow0 + h) * sh.nbm + j] = mb + logf(sb);
       }
     }
     __syncthreads();
@@ -206,6 +227,8 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         acc[h][k].y *= al[h];
       }
     }
+    const bool need_f16 = vprom || any_dense;
+    const bool need_i4 = MODE == 0 && !vprom && any_mixed;
 #pragma unroll
     for (int p = 0; p < NPASS; ++p) {
       const int tt = p * RPC + row;
@@ -213,27 +236,31 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
       float pw[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) pw[h] = S.pp[h][tt];
-      if (vprom) {
+      float2 vf[4];
+      if (need_f16) {
         const __half* vsrc = resid ? t.vres + u * st.res + (size_t)tt * D
                                    : t.v2 + u * st.tier2 + (tok0 + tt) * D;
         const uint4 vv = *reinterpret_cast<const uint4*>(vsrc + cl * 8);
         const __half2* vh = reinterpret_cast<const __half2*>(&vv);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 vf = __half22float2(vh[k]);
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            acc[h][k] = __ffma2_rn(make_float2(pw[h], pw[h]), vf, acc[h][k]);
-        }
-      } else {
+        for (int k = 0; k < 4; ++k) vf[k] = __half22float2(vh[k]);
+      }
+      float2 cf[4];
+      float2 meta = make_float2(0.f, 0.f);
+      if (need_i4) {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(
             t.vcodes + u * st.vcodes + ((size_t)j * BLK + tt) * (D / 2) + cl * 4);
-        const float2 meta = *reinterpret_cast<const float2*>(
+        meta = *reinterpret_cast<const float2*>(
             t.vmeta + u * st.vmeta + (((size_t)j * BLK + tt) * NG + (cl * 8) / VG) * 2);
-        float2 cf[4];
         u4x8_to_f2(w, cf);
+      }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < G; ++h) {
+        if (vprom || dh[h]) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            acc[h][k] = __ffma2_rn(make_float2(pw[h], pw[h]), vf[k], acc[h][k]);
+        } else {
           const float ws = pw[h] * meta.x;
           zacc[h] = fmaf(pw[h], meta.y, zacc[h]);
 #pragma unroll

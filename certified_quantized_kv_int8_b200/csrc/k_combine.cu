@@ -1,5 +1,6 @@
-// Split-K combine, value bound E_val, block-ranking consistency check and the
-// rung 3 / rung 4 decisions; and the combine of the dense fallback.
+// Block-ranking consistency check with the rung 3 / rung 4 decisions (before
+// the attention pass), split-K combine with the value bound E_val (after it),
+// and the combine of the dense passes from Tier 2.
 //
 // Runtime-Certified Bounded-Error Quantized Attention, Methodology §2
 // (E_val = sum over INT4-valued blocks of attention mass times eta_b) and §3
@@ -9,9 +10,10 @@
 //
 // Readings used: the check compares the ordered top-min(rank_r, |P|) lists of
 // promoted blocks by INT8 and by FP16 block log-mass (ties to the lower block
-// index); rung 3 also fires when E_key stayed above eps_key after widening or
-// when E_val > eps_val; rung 4 fires when at least need_dense =
-// ceil(layer_dense_frac * n_q_heads) heads of a (layer, batch row) took rung 3.
+// index); rung 3 also fires when E_key stayed above eps_key after widening;
+// rung 4 fires when at least need_dense = ceil(layer_dense_frac * n_q_heads)
+// heads of a (layer, batch row) took rung 3 that way.  After the attention
+// pass, a head whose E_val exceeds eps_val also takes rung 3 (post-check).
 #include "cqa_internal.cuh"
 
 namespace cqa {
@@ -44,11 +46,9 @@ __device__ KI next_best(const float* key, const uint8_t* bf, int nb, KI prev, in
   return best;
 }
 
-template <int D, int G>
-__global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, int need_dense, Scratch sc,
-                               float* __restrict__ out, float* __restrict__ e_key,
-                               float* __restrict__ e_val, uint8_t* __restrict__ rung) {
-  constexpr int CPL = D / 32;  // channels per lane
+// Rank check and the rung 3 / rung 4 decision, before the attention pass.
+// grid B, one warp per query head (looping when n_q_heads > 32).
+__global__ void decide_kernel(DecodeShape sh, cqa_thresholds th, int need_dense, Scratch sc) {
   __shared__ int n3;
   extern __shared__ uint8_t r3[];  // [Hq]
   const int b = blockIdx.x;
@@ -56,31 +56,10 @@ __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, int need_dense
   const bool naive = th.naive != 0;
   if (threadIdx.x == 0) n3 = 0;
   __syncthreads();
-
   for (int h = warp; h < sh.Hq; h += nwarp) {
-    const int g = h / G, hh = h - g * G;
+    const int g = h / sh.G;
     const int unit = b * sh.Hkv + g;
     const size_t row = (size_t)b * sh.Hq + h;
-    float M = -INFINITY;
-    for (int c = 0; c < sh.nchunks; ++c)
-      M = fmaxf(M, sc.part_s[(((size_t)unit * sc.max_chunks + c) * G + hh) * 3]);
-    float L = 0.f, E = 0.f, o[CPL];
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) o[k] = 0.f;
-    for (int c = 0; c < sh.nchunks; ++c) {
-      const size_t pi = ((size_t)unit * sc.max_chunks + c) * G + hh;
-      const float mc = sc.part_s[pi * 3];
-      const float w = mc == -INFINITY ? 0.f : expf(mc - M);
-      L += sc.part_s[pi * 3 + 1] * w;
-      E += sc.part_s[pi * 3 + 2] * w;
-#pragma unroll
-      for (int k = 0; k < CPL; ++k) o[k] += sc.part_o[pi * D + lane + 32 * k] * w;
-    }
-    const float inv = 1.f / L;
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) out[row * D + lane + 32 * k] = o[k] * inv;
-    const float ev = E * inv;
-
     uint8_t hf = sc.hflags[row];
     if (!naive) {
       const uint8_t* bf = sc.bflags + (size_t)unit * sh.nbm;
@@ -99,29 +78,105 @@ __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, int need_dense
         fail = p8.i != p16.i;
       }
       if (fail) hf |= HF_RANKFAIL;
-      if (ev > th.eps_val) hf |= HF_VALFAIL;
     }
-    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL | HF_VALFAIL));
+    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
     if (lane == 0) {
       sc.hflags[row] = hf;
-      e_key[row] = sc.ekey[row];
-      e_val[row] = ev;
-      rung[row] = (hf & HF_VALUE) ? 2 : ((hf & HF_WIDENED) ? 1 : 0);
       r3[h] = is3 ? 1 : 0;
       if (is3) atomicAdd(&n3, 1);
     }
   }
   __syncthreads();
   const bool layer = !naive && n3 >= need_dense;
-  for (int h = threadIdx.x; h < sh.Hq; h += blockDim.x) {
-    const size_t row = (size_t)b * sh.Hq + h;
-    const uint8_t dv = layer ? 4 : (r3[h] ? 3 : 0);
-    sc.dense[row] = dv;
-    if (dv) rung[row] = dv;
-  }
+  for (int h = threadIdx.x; h < sh.Hq; h += blockDim.x)
+    sc.dense[(size_t)b * sh.Hq + h] = layer ? 4 : (r3[h] ? 3 : 0);
 }
 
-// One warp per (batch row, query head); only dense heads are written.
+__device__ __forceinline__ float cwarp_max(float x) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
+  return x;
+}
+
+__device__ __forceinline__ float cwarp_sum(float x) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
+}
+
+// Merge the split-K partials of one head (a warp): returns o / L in o, and L, E.
+template <int D, int G>
+__device__ __forceinline__ void merge_head(const Scratch& sc, int nchunks, int unit, int hh,
+                                           int lane, float (&o)[D / 32], float& L, float& E) {
+  constexpr int CPL = D / 32;
+  const size_t base = (size_t)unit * sc.max_chunks * G + hh;  // partial index of chunk 0
+  float ml = -INFINITY;
+  for (int c = lane; c < nchunks; c += 32) ml = fmaxf(ml, sc.part_s[(base + (size_t)c * G) * 3]);
+  const float M = cwarp_max(ml);
+  float ll = 0.f, el = 0.f;
+  for (int c = lane; c < nchunks; c += 32) {
+    const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
+    const float w = ps[0] == -INFINITY ? 0.f : expf(ps[0] - M);
+    ll += ps[1] * w;
+    el += ps[2] * w;
+  }
+  L = cwarp_sum(ll);
+  E = cwarp_sum(el);
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) o[k] = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < nchunks; ++c) {
+    const size_t pi = base + (size_t)c * G;
+    const float mc = sc.part_s[pi * 3];
+    const float w = mc == -INFINITY ? 0.f : expf(mc - M);
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) o[k] += sc.part_o[pi * D + lane + 32 * k] * w;
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) o[k] *= inv;
+}
+
+// Outputs, E_val and the E_val post-check; one warp per (batch row, head).
+template <int D, int G>
+__global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
+                               float* __restrict__ out, float* __restrict__ e_key,
+                               float* __restrict__ e_val, uint8_t* __restrict__ rung) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // b * Hq + h
+  if (row >= sh.B * sh.Hq) return;
+  const int b = row / sh.Hq, h = row - b * sh.Hq;
+  const int g = h / G, hh = h - g * G;
+  float o[CPL], L, E;
+  merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, lane, o, L, E);
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) out[(size_t)row * D + lane + 32 * k] = o[k];
+  if (lane != 0) return;
+  const uint8_t dv = sc.dense[row];
+  uint8_t hf = sc.hflags[row];
+  const float ev = E / L;
+  if (dv) {
+    e_key[row] = 0.f;
+    e_val[row] = 0.f;
+    rung[row] = dv;
+  } else if (!th.naive && ev > th.eps_val) {
+    // post-check failure: exact attention follows in a separate dense pass
+    hf |= HF_VALFAIL;
+    sc.dense[row] = 3 | DENSE_LATE;
+    e_key[row] = 0.f;
+    e_val[row] = 0.f;
+    rung[row] = 3;
+  } else {
+    e_key[row] = sc.ekey[row];
+    e_val[row] = ev;
+    rung[row] = (hf & HF_VALUE) ? 2 : ((hf & HF_WIDENED) ? 1 : 0);
+  }
+  sc.hflags[row] = hf;
+}
+
+// One warp per (batch row, query head): heads recomputed by a dense pass
+// (all heads for cqa_dense_reference, DENSE_LATE heads otherwise).
 template <int D, int G>
 __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
                                      float* __restrict__ out, float* __restrict__ e_key,
@@ -130,41 +185,24 @@ __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
   const int row = blockIdx.x;  // b * Hq + h
   const int lane = threadIdx.x;
   const int b = row / sh.Hq, h = row - b * sh.Hq;
-  const uint8_t dv = all_heads ? 4 : sc.dense[row];
-  if (dv == 0) return;
+  if (!all_heads && !(sc.dense[row] & DENSE_LATE)) return;
   const int g = h / G, hh = h - g * G;
-  const int unit = b * sh.Hkv + g;
-  float M = -INFINITY;
-  for (int c = 0; c < sh.nchunks; ++c)
-    M = fmaxf(M, sc.part_s[(((size_t)unit * sc.max_chunks + c) * G + hh) * 3]);
-  float L = 0.f, o[CPL];
+  float o[CPL], L, E;
+  merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, lane, o, L, E);
 #pragma unroll
-  for (int k = 0; k < CPL; ++k) o[k] = 0.f;
-  for (int c = 0; c < sh.nchunks; ++c) {
-    const size_t pi = ((size_t)unit * sc.max_chunks + c) * G + hh;
-    const float mc = sc.part_s[pi * 3];
-    const float w = mc == -INFINITY ? 0.f : expf(mc - M);
-    L += sc.part_s[pi * 3 + 1] * w;
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) o[k] += sc.part_o[pi * D + lane + 32 * k] * w;
-  }
-  const float inv = 1.f / L;
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) out[(size_t)row * D + lane + 32 * k] = o[k] * inv;
+  for (int k = 0; k < CPL; ++k) out[(size_t)row * D + lane + 32 * k] = o[k];
   if (!all_heads && lane == 0) {
     e_key[row] = 0.f;
     e_val[row] = 0.f;
-    rung[row] = dv;
+    rung[row] = 3;
   }
 }
 
 template <int D, int G>
-cudaError_t combine_t(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
-                      const Scratch& sc, float* out, float* e_key, float* e_val, uint8_t* rung,
-                      cudaStream_t s) {
-  const int threads = 32 * (sh.Hq < 32 ? sh.Hq : 32);
-  combine_kernel<D, G><<<sh.B, threads, sh.Hq, s>>>(sh, th, need_dense, sc, out, e_key, e_val,
-                                                    rung);
+cudaError_t combine_t(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
+                      float* out, float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
+  const int rows = sh.B * sh.Hq;
+  combine_kernel<D, G><<<(rows + 7) / 8, 256, 0, s>>>(sh, th, sc, out, e_key, e_val, rung);
   return cudaGetLastError();
 }
 
@@ -197,10 +235,17 @@ cudaError_t dense_combine_t(const DecodeShape& sh, const Scratch& sc, int all_he
     return cudaErrorInvalidValue;                                  \
   } while (0)
 
-cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
-                           const Scratch& sc, float* out, float* e_key, float* e_val,
-                           uint8_t* rung, cudaStream_t s) {
-  CQA_DISPATCH_DG(combine_t, sh, th, need_dense, sc, out, e_key, e_val, rung, s);
+cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
+                           float* out, float* e_key, float* e_val, uint8_t* rung,
+                           cudaStream_t s) {
+  CQA_DISPATCH_DG(combine_t, sh, th, sc, out, e_key, e_val, rung, s);
+}
+
+cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
+                          const Scratch& sc, cudaStream_t s) {
+  const int threads = 32 * (sh.Hq < 32 ? sh.Hq : 32);
+  decide_kernel<<<sh.B, threads, sh.Hq, s>>>(sh, th, need_dense, sc);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_dense_combine(const DecodeShape& sh, const Scratch& sc, int all_heads,

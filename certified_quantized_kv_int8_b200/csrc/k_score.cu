@@ -84,7 +84,10 @@ __global__ void __launch_bounds__(WARPS * 32, 3)
   __shared__ __align__(16) float lg[WARPS][G][BLK];
   const int nw = gridDim.x * WARPS;
 
-  for (int it = blockIdx.x * WARPS + wib; it < n_items; it += nw) {
+  const int n_res = n_items - n_sealed;
+  for (int it0 = blockIdx.x * WARPS + wib; it0 < n_items; it0 += nw) {
+    // the residual items (one per unit) go first so they overlap the blocks
+    const int it = it0 < n_res ? n_sealed + it0 : it0 - n_res;
     if (it < n_sealed) {
       const int unit = it / sh.nb, j = it - unit * sh.nb;
       const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
@@ -177,42 +180,65 @@ __global__ void __launch_bounds__(WARPS * 32, 3)
       }
       __syncwarp();
     } else {
-      // residual block: exact logits from the FP16 keys kept in device memory
+      // residual block: exact logits from the FP16 keys kept in device memory;
+      // LPR lanes per token row, 8 channels each
+      constexpr int LPR = D / 8;
+      constexpr int RW = 32 / LPR;  // rows per warp pass
       const int unit = it - n_sealed;
       const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
       const size_t u = (size_t)unit0 + unit;
+      const int cl = lane % LPR, rl = lane / LPR;
       const __half* kr = t.kres + u * st.res;
+      float2 qf[G][4];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(
+            q + ((size_t)b * sh.Hq + (size_t)g * G + h) * D + cl * 8));
+        const __half2* qh = reinterpret_cast<const __half2*>(&qv);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qf[h][k] = __half22float2(qh[k]);
+      }
+      for (int r0 = 0; r0 < sh.r; r0 += RW) {
+        const int tok = r0 + rl;
+        float2 kf[4];
+        if (tok < sh.r) {
+          const uint4 kv = *reinterpret_cast<const uint4*>(kr + (size_t)tok * D + cl * 8);
+          const __half2* kh = reinterpret_cast<const __half2*>(&kv);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) kf[k] = __half22float2(kh[k]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) kf[k] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) a = __ffma2_rn(qf[h][k], kf[k], a);
+          float v = a.x + a.y;
+#pragma unroll
+          for (int m = LPR / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+          if (cl == 0 && tok < sh.r) lg[wib][h][tok] = v * sh.sigma;
+        }
+      }
+      __syncwarp();
 #pragma unroll 1
       for (int h = 0; h < G; ++h) {
-        const __half* qh = q + ((size_t)b * sh.Hq + (size_t)g * G + h) * D;
-        float x[2];
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const int tok = lane + 32 * tt;
-          float acc = -INFINITY;
-          if (tok < sh.r) {
-            acc = 0.f;
-            for (int c = 0; c < D; c += 2) {
-              const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(kr + tok * D + c));
-              const float2 qf = __half22float2(*reinterpret_cast<const __half2*>(qh + c));
-              acc = fmaf(qf.x, kf.x, acc);
-              acc = fmaf(qf.y, kf.y, acc);
-            }
-            acc *= sh.sigma;
-            sc.logits[((size_t)b * sh.Hq + (size_t)g * G + h) * sc.ls + (size_t)sh.nb * BLK + tok] =
-                acc;
-          }
-          x[tt] = acc;
-        }
-        const float m = warp_max(fmaxf(x[0], x[1]));
+        const float x0 = lane < sh.r ? lg[wib][h][lane] : -INFINITY;
+        const float x1 = lane + 32 < sh.r ? lg[wib][h][lane + 32] : -INFINITY;
+        float* lo = sc.logits + ((size_t)b * sh.Hq + (size_t)g * G + h) * sc.ls + (size_t)sh.nb * BLK;
+        if (lane < sh.r) lo[lane] = x0;
+        if (lane + 32 < sh.r) lo[lane + 32] = x1;
         float lse = -INFINITY;
         if (sh.r > 0) {
-          const float ssum = warp_sum((x[0] > -INFINITY ? expf(x[0] - m) : 0.f) +
-                                      (x[1] > -INFINITY ? expf(x[1] - m) : 0.f));
+          const float m = warp_max(fmaxf(x0, x1));
+          const float ssum = warp_sum((x0 > -INFINITY ? expf(x0 - m) : 0.f) +
+                                      (x1 > -INFINITY ? expf(x1 - m) : 0.f));
           lse = m + logf(ssum);
         }
         if (lane == 0) sc.ell_res[(size_t)b * sh.Hq + (size_t)g * G + h] = lse;
       }
+      __syncwarp();
     }
   }
 }

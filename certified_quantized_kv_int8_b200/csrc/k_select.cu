@@ -18,6 +18,10 @@
 //   E_key = min(tanh(dT/2), m_ub (e^(2 dT) - 1)), 0 when T is empty.
 // Heads with E_key > eps_key double K* (at most max_expand times).
 // A block's FP16 values are promoted when some head has m8_b * eta_b > v_tol.
+//
+// The CTA's 1024 threads form G groups, one per query head; the per-head
+// work (log-sum-exp, sort, scan, tail reductions) synchronises each group on
+// its own named barrier, and only the union steps use the whole CTA.
 #include "cqa_internal.cuh"
 
 namespace cqa {
@@ -25,7 +29,6 @@ namespace cqa {
 namespace {
 
 constexpr int THREADS = 1024;
-constexpr int NWARP = THREADS / 32;
 
 __device__ __forceinline__ uint64_t sort_key(float ell, uint32_t idx) {
   const float f = __fadd_rn(ell, 0.0f);  // one zero
@@ -34,38 +37,50 @@ __device__ __forceinline__ uint64_t sort_key(float ell, uint32_t idx) {
   return ((uint64_t)(~ord) << 32) | idx;  // ascending = ell descending, then index ascending
 }
 
-__device__ __forceinline__ float block_max(float x, float* red) {
-  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) red[w] = x;
-  __syncthreads();
-  x = l < NWARP ? red[l] : -INFINITY;
-  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
+__device__ __forceinline__ void group_bar(int grp, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(grp + 1), "r"(nthreads) : "memory");
+}
+
+template <class T>
+__device__ __forceinline__ T wmax(T x) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) {
+    const T y = __shfl_xor_sync(0xffffffffu, x, m);
+    x = x > y ? x : y;
+  }
   return x;
 }
 
-__device__ __forceinline__ double block_sum(double x, double* red) {
-  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) red[w] = x;
-  __syncthreads();
-  x = l < NWARP ? red[l] : 0.0;
+template <class T>
+__device__ __forceinline__ T wsum(T x) {
+#pragma unroll
   for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
   return x;
 }
 
-__device__ __forceinline__ int block_count(int x, int* red) {
-  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) red[w] = x;
-  __syncthreads();
-  x = l < NWARP ? red[l] : 0;
-  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
-  return x;
-}
+// Reductions over one thread group (nw warps) through a per-group slot array.
+struct Group {
+  int id, nthreads, nw, wig, lane, tig;
+  template <class T>
+  __device__ T max(T x, T* slot, T ident) const {
+    x = wmax(x);
+    group_bar(id, nthreads);
+    if (lane == 0) slot[wig] = x;
+    group_bar(id, nthreads);
+    x = lane < nw ? slot[lane] : ident;
+    return wmax(x);
+  }
+  template <class T>
+  __device__ T sum(T x, T* slot) const {
+    x = wsum(x);
+    group_bar(id, nthreads);
+    if (lane == 0) slot[wig] = x;
+    group_bar(id, nthreads);
+    x = lane < nw ? slot[lane] : T(0);
+    return wsum(x);
+  }
+  __device__ void sync() const { group_bar(id, nthreads); }
+};
 
 __device__ double e_key_bound(double dT, double dA, double m8T) {
   const double a = m8T * exp(dT);
@@ -80,175 +95,165 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
                                                          Scratch sc, int NP) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int nb = sh.nb;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
-  float* mass = reinterpret_cast<float*>(keys + (size_t)G * NP);
-  uint8_t* pflag = reinterpret_cast<uint8_t*>(mass + (size_t)G * nb);
+  uint64_t* keys_all = reinterpret_cast<uint64_t*>(smem);
+  float* mass_all = reinterpret_cast<float*>(keys_all + (size_t)G * NP);
+  uint8_t* pflag = reinterpret_cast<uint8_t*>(mass_all + (size_t)G * nb);
   uint8_t* vflag = pflag + nb;
-  __shared__ double redd[NWARP];
-  __shared__ float redf[NWARP];
-  __shared__ int redi[NWARP];
-  __shared__ float lse_s[G], mres_s[G], dA_s[G];
+  constexpr int GT = THREADS / G;  // threads per head group
+  __shared__ double slot_d[G][32];
+  __shared__ float slot_f[G][32];
+  __shared__ int slot_i[G][32];
   __shared__ int kst[G], kold[G];
   __shared__ double ekey_s[G];
   __shared__ int any_fail;
+  __shared__ int npro_s;
   __shared__ unsigned hf_s[G];
 
   const int unit = blockIdx.x;
   const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
   const size_t u = (size_t)unit0 + unit;
-  const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;  // first query head of the group
-  const float* eta = t.eta + u * st.eta;
+  const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
   const int tid = threadIdx.x;
   const bool naive = th.naive != 0;
+  Group grp;
+  grp.id = tid / GT;
+  grp.nthreads = GT;
+  grp.nw = GT / 32;
+  grp.tig = tid - grp.id * GT;
+  grp.wig = grp.tig >> 5;
+  grp.lane = tid & 31;
+  const int h = grp.id;  // this group's head
+  const int tg = grp.tig;
+  uint64_t* keys = keys_all + (size_t)h * NP;
+  float* mass = mass_all + (size_t)h * nb;
+  const float* e8 = sc.ell8 + (hrow0 + h) * sh.nbm;
+  const float* dl = sc.delta + (hrow0 + h) * sh.nbm;
 
   for (int j = tid; j < nb; j += THREADS) {
     pflag[j] = 0;
     vflag[j] = 0;
   }
   if (tid < G) hf_s[tid] = 0;
+  if (tid == 0) npro_s = 0;
 
-  // log-sum-exp per head, masses, Delta max
-  for (int h = 0; h < G; ++h) {
-    const float* e8 = sc.ell8 + (hrow0 + h) * sh.nbm;
-    const float* dl = sc.delta + (hrow0 + h) * sh.nbm;
-    const float eres = sc.ell_res[hrow0 + h];
-    float mx = eres, dmax = 0.f;
-    for (int j = tid; j < nb; j += THREADS) {
-      mx = fmaxf(mx, e8[j]);
-      dmax = fmaxf(dmax, dl[j]);
-    }
-    mx = block_max(mx, redf);
-    dmax = block_max(dmax, redf);
-    double ssum = 0.0;
-    for (int j = tid; j < nb; j += THREADS) ssum += (double)expf(e8[j] - mx);
-    if (tid == 0 && eres > -INFINITY) ssum += (double)expf(eres - mx);
-    ssum = block_sum(ssum, redd);
-    const float lse = mx + (float)log(ssum);
-    for (int j = tid; j < nb; j += THREADS) mass[h * nb + j] = expf(e8[j] - lse);
-    for (int i = tid; i < NP; i += THREADS)
-      keys[(size_t)h * NP + i] = i < nb ? sort_key(e8[i], (uint32_t)i) : ~0ull;
-    if (tid == 0) {
-      lse_s[h] = lse;
-      mres_s[h] = eres > -INFINITY ? expf(eres - lse) : 0.f;
-      dA_s[h] = dmax;
-    }
+  // ---- per head: log-sum-exp, masses, Delta max, sort keys ----
+  const float eres = sc.ell_res[hrow0 + h];
+  float mx = eres, dmax = 0.f;
+  for (int j = tg; j < nb; j += GT) {
+    mx = fmaxf(mx, e8[j]);
+    dmax = fmaxf(dmax, dl[j]);
   }
-  __syncthreads();
+  mx = grp.max(mx, slot_f[h], -INFINITY);
+  const float dA = grp.max(dmax, slot_f[h], 0.f);
+  double ssum = 0.0;
+  for (int j = tg; j < nb; j += GT) ssum += (double)expf(e8[j] - mx);
+  if (tg == 0 && eres > -INFINITY) ssum += (double)expf(eres - mx);
+  ssum = grp.sum(ssum, slot_d[h]);
+  const float lse = mx + (float)log(ssum);
+  for (int j = tg; j < nb; j += GT) mass[j] = expf(e8[j] - lse);
+  for (int i = tg; i < NP; i += GT) keys[i] = i < nb ? sort_key(e8[i], (uint32_t)i) : ~0ull;
+  const float m_res_f = eres > -INFINITY ? expf(eres - lse) : 0.f;
+  grp.sync();
 
-  // bitonic sort of the G segments of NP keys each
+  // ---- bitonic sort of this head's NP keys ----
   const int half = NP >> 1;
   for (int k = 2; k <= NP; k <<= 1) {
     for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int p = tid; p < G * half; p += THREADS) {
-        const int seg = p / half, i = p - seg * half;
-        const int a = 2 * jj * (i / jj) + (i % jj);
+      for (int p = tg; p < half; p += GT) {
+        const int a = 2 * jj * (p / jj) + (p % jj);
         const int c = a + jj;
-        uint64_t* kk = keys + (size_t)seg * NP;
-        const uint64_t x = kk[a], y = kk[c];
+        const uint64_t x = keys[a], y = keys[c];
         const bool up = (a & k) == 0;
         if ((x > y) == up) {
-          kk[a] = y;
-          kk[c] = x;
+          keys[a] = y;
+          keys[c] = x;
         }
       }
-      __syncthreads();
+      grp.sync();
     }
   }
 
-  // K* per head: float64 inclusive scan of the sorted masses
-  const int per = (nb + THREADS - 1) / THREADS;
-  for (int h = 0; h < G; ++h) {
-    int kstar = 0;
-    if (naive) {
-      kstar = 0;
-    } else if (th.tau_cov >= 1.0f) {
-      kstar = nb;
-    } else {
-      const double tau = (double)th.tau_cov;
-      const double m_res = (double)mres_s[h];
-      const uint64_t* kk = keys + (size_t)h * NP;
-      const int i0 = tid * per, i1 = min(nb, i0 + per);
-      double local = 0.0;
-      for (int i = i0; i < i1; ++i) local += (double)mass[h * nb + (int)(kk[i] & 0xffffffffu)];
-      // exclusive scan of thread totals
-      const int l = tid & 31, w = tid >> 5;
-      double incl = local;
-      for (int m = 1; m < 32; m <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, incl, m);
-        if (l >= m) incl += y;
-      }
-      __syncthreads();
-      if (l == 31) redd[w] = incl;
-      __syncthreads();
-      double wbase = 0.0;
-      for (int x = 0; x < w; ++x) wbase += redd[x];
-      double run = m_res + wbase + (incl - local);
-      int cnt = 0;
-      for (int i = i0; i < i1; ++i) {
-        run += (double)mass[h * nb + (int)(kk[i] & 0xffffffffu)];
-        cnt += run < tau ? 1 : 0;  // prefix of i + 1 blocks below tau
-      }
-      cnt = block_count(cnt, redi);
-      // prefixes of 0..nb blocks below tau: the empty prefix plus cnt
-      kstar = (m_res < tau) ? min(nb, cnt + 1) : 0;
+  // ---- K*: float64 inclusive scan of the sorted masses ----
+  int kstar = 0;
+  if (naive) {
+    kstar = 0;
+  } else if (th.tau_cov >= 1.0f) {
+    kstar = nb;
+  } else {
+    const double tau = (double)th.tau_cov;
+    const double m_res = (double)m_res_f;
+    const int per = (nb + GT - 1) / GT;
+    const int i0 = tg * per, i1 = min(nb, i0 + per);
+    double local = 0.0;
+    for (int i = i0; i < i1; ++i) local += (double)mass[(int)(keys[i] & 0xffffffffu)];
+    double incl = local;
+    for (int m = 1; m < 32; m <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, m);
+      if (grp.lane >= m) incl += y;
     }
-    if (tid == 0) kst[h] = kstar;
-    __syncthreads();
+    grp.sync();
+    if (grp.lane == 31) slot_d[h][grp.wig] = incl;
+    grp.sync();
+    double wbase = 0.0;
+    for (int x = 0; x < grp.wig; ++x) wbase += slot_d[h][x];
+    double run = m_res + wbase + (incl - local);
+    int cnt = 0;
+    for (int i = i0; i < i1; ++i) {
+      run += (double)mass[(int)(keys[i] & 0xffffffffu)];
+      cnt += run < tau ? 1 : 0;  // prefix of i + 1 blocks below tau
+    }
+    cnt = grp.sum(cnt, slot_i[h]);
+    // prefixes of 0..nb blocks below tau: the empty prefix plus cnt
+    kstar = (m_res < tau) ? min(nb, cnt + 1) : 0;
   }
-
-  // mark the initial promoted set
-  for (int h = 0; h < G; ++h)
-    for (int i = tid; i < kst[h]; i += THREADS) pflag[(int)(keys[(size_t)h * NP + i] & 0xffffffffu)] = 1;
+  if (tg == 0) kst[h] = kstar;
+  for (int i = tg; i < kstar; i += GT) pflag[(int)(keys[i] & 0xffffffffu)] = 1;
   __syncthreads();
 
-  // E_key and rung-1 widening
+  // ---- E_key and rung-1 widening ----
   for (int round = 0;; ++round) {
-    for (int h = 0; h < G; ++h) {
-      const float* dl = sc.delta + (hrow0 + h) * sh.nbm;
-      float dT = 0.f;
-      double m8T = 0.0;
-      int ntail = 0;
-      for (int j = tid; j < nb; j += THREADS) {
-        if (!pflag[j]) {
-          dT = fmaxf(dT, dl[j]);
-          m8T += (double)mass[h * nb + j];
-          ++ntail;
-        }
+    float dT = 0.f;
+    double m8T = 0.0;
+    int ntail = 0;
+    for (int j = tg; j < nb; j += GT) {
+      if (!pflag[j]) {
+        dT = fmaxf(dT, dl[j]);
+        m8T += (double)mass[j];
+        ++ntail;
       }
-      dT = block_max(dT, redf);
-      m8T = block_sum(m8T, redd);
-      ntail = block_count(ntail, redi);
-      if (tid == 0) ekey_s[h] = ntail ? e_key_bound((double)dT, (double)dA_s[h], m8T) : 0.0;
     }
+    dT = grp.max(dT, slot_f[h], 0.f);
+    m8T = grp.sum(m8T, slot_d[h]);
+    ntail = grp.sum(ntail, slot_i[h]);
+    if (tg == 0) ekey_s[h] = ntail ? e_key_bound((double)dT, (double)dA, m8T) : 0.0;
     __syncthreads();
     if (tid == 0) {
       any_fail = 0;
-      for (int h = 0; h < G; ++h) {
-        kold[h] = kst[h];
-        if (!naive && ekey_s[h] > (double)th.eps_key && round < th.max_expand) {
-          kst[h] = min(nb, max(1, 2 * kst[h]));
-          hf_s[h] |= HF_WIDENED;
+      for (int hh = 0; hh < G; ++hh) {
+        kold[hh] = kst[hh];
+        if (!naive && ekey_s[hh] > (double)th.eps_key && round < th.max_expand) {
+          kst[hh] = min(nb, max(1, 2 * kst[hh]));
+          hf_s[hh] |= HF_WIDENED;
           any_fail = 1;
         }
       }
     }
     __syncthreads();
     if (!any_fail) break;
-    for (int h = 0; h < G; ++h)
-      for (int i = kold[h] + tid; i < kst[h]; i += THREADS)
-        pflag[(int)(keys[(size_t)h * NP + i] & 0xffffffffu)] = 1;
+    for (int i = kold[h] + tg; i < kst[h]; i += GT) pflag[(int)(keys[i] & 0xffffffffu)] = 1;
     __syncthreads();
   }
 
-  // rung 2: value promotion
+  // ---- rung 2: value promotion ----
+  const float* eta = t.eta + u * st.eta;
   if (!naive) {
     for (int j = tid; j < nb; j += THREADS) {
       const float e = eta[j];
       uint8_t vp = 0;
-      for (int h = 0; h < G; ++h) {
-        if (mass[h * nb + j] * e > th.v_tol) {
+      for (int hh = 0; hh < G; ++hh) {
+        if (mass_all[(size_t)hh * nb + j] * e > th.v_tol) {
           vp = 1;
-          atomicOr(&hf_s[h], (unsigned)HF_VALUE);
+          atomicOr(&hf_s[hh], (unsigned)HF_VALUE);
         }
       }
       vflag[j] = vp;
@@ -257,15 +262,23 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
   __syncthreads();
 
   uint8_t* bf = sc.bflags + ((size_t)b * sh.Hkv + g) * sh.nbm;
-  for (int j = tid; j < nb; j += THREADS)
+  int npro = 0;
+  for (int j = tid; j < nb; j += THREADS) {
     bf[j] = (pflag[j] ? BF_KEY : 0) | (vflag[j] ? BF_VAL : 0);
+    npro += pflag[j] ? 1 : 0;
+  }
+  // promoted-block count of the unit, for the host's key-prefetch policy
+  npro = wsum(npro);
+  if (grp.lane == 0 && npro) atomicAdd(&npro_s, npro);
+  __syncthreads();
+  if (tid == 0 && sc.promo) sc.promo[u] = npro_s;
   if (tid < G) {
-    const int h = tid;
-    unsigned f = hf_s[h];
-    if (!naive && ekey_s[h] > (double)th.eps_key) f |= HF_KEYFAIL;
-    sc.hflags[hrow0 + h] = (uint8_t)f;
-    sc.kstar[hrow0 + h] = kst[h];
-    sc.ekey[hrow0 + h] = (float)ekey_s[h];
+    const int hh = tid;
+    unsigned f = hf_s[hh];
+    if (!naive && ekey_s[hh] > (double)th.eps_key) f |= HF_KEYFAIL;
+    sc.hflags[hrow0 + hh] = (uint8_t)f;
+    sc.kstar[hrow0 + hh] = kst[hh];
+    sc.ekey[hrow0 + hh] = (float)ekey_s[hh];
   }
 }
 

@@ -101,7 +101,8 @@ typedef struct cqa_trace {
 
 /* Allocate both tiers for `cfg` on cfg->device: Tier 1 and scratch in device
  * memory, Tier 2 (n_layers * batch * n_kv_heads * max_ctx * head_dim * 2 fp16)
- * in pinned, device-mapped host memory.  *out receives the handle. */
+ * in pinned, device-mapped host memory, and the two key-staging buffers of
+ * cqa_set_key_prefetch.  *out receives the handle. */
 int cqa_cache_create(const cqa_config* cfg, cqa_cache** out);
 
 /* Free everything the cache owns (synchronises the device first).  NULL is a no-op. */
@@ -169,6 +170,21 @@ enum {
 };
 int64_t cqa_debug_export(cqa_cache* cache, int layer, int what, void* host_dst, size_t bytes);
 
+/* Whole-layer key prefetch.  Promotion reads the FP16 keys of the selected
+ * blocks from Tier 2.  When a layer's last decode promoted nearly all of its
+ * blocks, copying the layer's sealed keys to device memory with the copy
+ * engine is faster than gathering them block by block, and the copy of the
+ * next layer can run while the current layer computes.  With mode 1
+ * (adaptive, the default) cqa_decode of layer l stages layer l and layer
+ * (l + 1) % n_layers whenever their last decode promoted at least
+ * min_fraction of their blocks (the first decode of a layer never does);
+ * mode 2 always stages; mode 0 never does.  Staging changes no result: the
+ * promoted keys are the same bytes, and blocks the copy did not cover are
+ * read from Tier 2 as before.  It uses two device buffers of one layer's
+ * keys each (batch * n_kv_heads * max_ctx * head_dim fp16), allocated by
+ * cqa_cache_create, and a copy stream owned by the cache. */
+int cqa_set_key_prefetch(cqa_cache* cache, int mode, float min_fraction);
+
 /* Per-phase device time of the library's kernels (tracing).  Between
  * cqa_profile_begin and cqa_profile_end, every kernel the cache launches is
  * bracketed by two CUDA events recorded on the call's stream; end waits for
@@ -179,11 +195,15 @@ enum {
   CQA_PHASE_APPEND_TAIL = 1,   /* Tier-2 copy, residual block, value ranges */
   CQA_PHASE_SCORE = 2,         /* INT8 scoring pass */
   CQA_PHASE_SELECT = 3,        /* coverage selection, E_key, rungs 1-2 */
-  CQA_PHASE_ATTEND = 4,        /* split-K attention with fused promotion */
-  CQA_PHASE_COMBINE = 5,       /* combine, E_val, rank check, rungs 3-4 */
-  CQA_PHASE_DENSE_ATTEND = 6,  /* exact attention of dense-fallback heads */
-  CQA_PHASE_DENSE_COMBINE = 7, /* combine of the dense fallback */
-  CQA_PHASE_COUNT = 8
+  CQA_PHASE_PROMOTE = 4,       /* FP16 keys of promoted blocks from Tier 2: exact logits */
+  CQA_PHASE_DECIDE = 5,        /* rank check, rungs 3-4 */
+  CQA_PHASE_DENSE_KEYS = 6,    /* exact logits of not-promoted blocks for dense heads */
+  CQA_PHASE_ATTEND = 7,        /* split-K softmax and P.V, value bound */
+  CQA_PHASE_COMBINE = 8,       /* split-K combine, E_val */
+  CQA_PHASE_DENSE_ATTEND = 9,  /* exact attention from Tier 2 (E_val post-check, reference) */
+  CQA_PHASE_DENSE_COMBINE = 10,
+  CQA_PHASE_PREFETCH = 11,     /* copy-engine copy of a layer's Tier-2 keys (not a kernel) */
+  CQA_PHASE_COUNT = 12
 };
 /* Start (or restart) profiling; max_launches bounds the recorded launches
  * (further launches are counted but not timed). */

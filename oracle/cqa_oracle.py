@@ -364,9 +364,11 @@ def decode(q16: np.ndarray, units: list, th: Thresholds) -> dict:
     3 per-head dense, 4 whole-layer dense), layer_dense, and per-group traces.
 
     Rung 3 fires when a head's E_key stays above eps_key after max_expand
-    widenings, when its rank check fails, or when E_val > eps_val.  Rung 4
-    (whole layer dense) fires when at least ceil(layer_dense_frac * H_q) heads
-    of the layer took rung 3.  Dense heads return O_dense with E_key = E_val = 0.
+    widenings or when its rank check fails.  Rung 4 (whole layer dense) fires
+    when at least ceil(layer_dense_frac * H_q) heads of the layer took rung 3
+    that way.  Otherwise a head whose E_val exceeds eps_val also takes rung 3
+    (a post-check; it does not re-count rung 4).  Dense heads return O_dense
+    with E_key = E_val = 0.
     """
     Hq, d = q16.shape
     Hkv = len(units)
@@ -375,14 +377,17 @@ def decode(q16: np.ndarray, units: list, th: Thresholds) -> dict:
     out = np.concatenate([g["out"] for g in groups])
     e_key = np.concatenate([g["e_key"] for g in groups])
     e_val = np.concatenate([g["e_val"] for g in groups])
+    # rungs 3 and 4 are decided before the attention pass, from the E_key and
+    # rank-check failures; the E_val post-check (eps_val) then sends single
+    # heads to dense attention without re-counting rung 4
     rung3 = np.concatenate([g["key_fail"] | g["rank_fail"] for g in groups])
-    if not th.naive:
-        rung3 |= e_val > th.eps_val
     rung = np.zeros(Hq, np.uint8)
     rung[np.concatenate([g["expanded"] for g in groups])] = 1
     rung[np.concatenate([g["rung2"] for g in groups])] = 2
     need = math.ceil(th.layer_dense_frac * Hq)
     layer_dense = (not th.naive) and int(rung3.sum()) >= need
+    if not th.naive and not layer_dense:
+        rung3 = rung3 | (e_val > th.eps_val)
     dense_heads = np.ones(Hq, bool) if layer_dense else rung3
     for h in np.nonzero(dense_heads)[0]:
         u = units[h // G]

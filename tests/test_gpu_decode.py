@@ -51,6 +51,8 @@ TINY_TH = {
     "head_dense": dict(tau_cov=0.3, eps_key=-1.0, max_expand=0),
     "layer_dense": dict(layer_dense_frac=0.0),
     "rank2": dict(rank_r=2, tau_cov=0.8),
+    "val_post_check": dict(tau_cov=0.9, eps_val=0.17),
+    "val_post_check_tight": dict(eps_val=0.0),
 }
 
 
@@ -91,8 +93,11 @@ def test_full_promotion_equals_dense_reference(cqa):
         torch.cuda.synchronize()
         assert np.all(ek.cpu().numpy() == 0) and np.all(ev.cpu().numpy() == 0)
         assert np.abs(out.cpu().numpy() - dense).max() <= 1e-5
-        forced = cache.decode(0, q, cqa.Thresholds(layer_dense_frac=0.0))[0].cpu().numpy()
-        assert np.array_equal(forced, dense)
+        forced, fk, fv, frung = cache.decode(0, q, cqa.Thresholds(layer_dense_frac=0.0))
+        torch.cuda.synchronize()
+        assert np.all(frung.cpu().numpy() == 4) and np.all(fk.cpu().numpy() == 0)
+        # the forced whole-layer fallback is exact attention (float32 rounding apart)
+        assert np.abs(forced.cpu().numpy() - dense).max() <= 1e-5
         K, V = sk.kv_layer(w, 0, 0, ctx, "cpu")
         qc = q.cpu().numpy()[0]
         G = w.group
@@ -156,3 +161,31 @@ def test_appended_steps_match_oracle(cqa):
                 compare_decode(row(res, 0), ora, oracle_thresholds(th), w.group, log,
                                label=f"step {step}")
     assert len(log.entries) <= 1
+
+
+def test_key_prefetch_changes_no_result(cqa):
+    """Staging a layer's keys with the copy engine gives bit-identical decodes,
+    across appends that seal new blocks between the copy and its use."""
+    w = sk.WORKLOADS["llama8b_8k_1layer"]
+    ctx = 4096 + 60
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    results = {}
+    for mode in (0, 2, 1):
+        with cqa.Cache(2, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx + 16) as cache:
+            cache.set_key_prefetch(mode, 0.5)
+            fill_cache(cache, w, [0, 1], ctx)
+            outs = []
+            for step in range(3):
+                for layer in (0, 1):
+                    t = ctx + 4 * step
+                    K, V = sk.kv_layer(w, layer, t, t + 4, "cuda")  # seals a block at step 1
+                    cache.append(layer, K, V)
+                    q = sk.queries(w, layer, step, "cuda")
+                    o = cache.decode(layer, q, th)
+                    torch.cuda.synchronize()
+                    outs.append([x.cpu().numpy() for x in o])
+            results[mode] = outs
+    for mode in (2, 1):
+        for a, b in zip(results[0], results[mode]):
+            for x, y in zip(a, b):
+                assert np.array_equal(x, y), f"prefetch mode {mode} changed a result"
