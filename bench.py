@@ -298,16 +298,18 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
                 cache.append(layer, kv[layer][0], kv[layer][1], stream)
             cache.decode(layer, qs[layer], thr, outputs=outs, stream=stream)
 
-    def timed(first, n, thr, profile=False):
+    def timed(first, n, thr, profile=False, label="timed"):
         barrier(dist, device)
         torch.cuda.synchronize(device)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if profile:
             cache.profile_begin(1 << 20)
+        torch.cuda.nvtx.range_push(label)  # lets a profiler select the timed steps
         a.record(stream)
         for s in range(first, first + n):
             run_step(s, thr)
         b.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(device)
         prof = cache.profile_end() if profile else None
         barrier(dist, device)
@@ -365,7 +367,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
 
     # the INT8/INT4 path alone (certification off): effective KV GB/s
     first = args.warmup + args.steps + n_e2e
-    n_el, nprof = timed(first, n_naive, th_naive, profile=True)
+    n_el, nprof = timed(first, n_naive, th_naive, profile=True, label="int8_int4")
     n_max = max_over_ranks(n_el, dist, device)
     nb_total = sum(cache.length(layer) // BLOCK for layer in range(L))
     t1_bytes = nb_total * B * Hkv * tier1_bytes_per_block(d)  # per step (lengths at the end)
@@ -452,6 +454,8 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "tier1_bytes_per_step": t1_bytes,
             "kernel_ms_per_step": quant_ms,
             "kernel_kv_gbs": t1_bytes / (quant_ms * 1e-3) / 1e9,
+            "phases_ms_per_step": {k: v / n_naive for k, v in nphase_ms.items() if nphase_n[k]},
+            "launches_per_step": {k: v / n_naive for k, v in nphase_n.items() if v},
         },
         "promotion": {
             "key_promoted_frac": frac_k, "value_promoted_frac": frac_v,
@@ -565,12 +569,17 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(sk.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode only the first N layers (profiling captures; the reported "
+                         "line then covers N layers, not the workload's step)")
     ap.add_argument("--clocks-csv", default=None,
                     help="keep the nvidia-smi samples of the timed region in this file")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = sk.WORKLOADS[args.workload]
+    if args.layers is not None:
+        w = dataclasses.replace(w, n_layers=max(1, min(args.layers, w.n_layers)))
     ws, rank, local = dist_env()
 
     if args.impl == "reference":

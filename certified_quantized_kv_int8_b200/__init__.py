@@ -30,7 +30,7 @@ __all__ = [
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "PHASES", "cqa_dense_attention_noalloc",
-    "cqa_set_key_prefetch",
+    "cqa_set_key_prefetch", "cqa_device_status",
     "EXPORT_KCODES", "EXPORT_KSCALE", "EXPORT_VCODES", "EXPORT_VMETA", "EXPORT_ETA",
     "EXPORT_VRANGE", "EXPORT_RESIDUAL", "EXPORT_TIER2",
 ]
@@ -42,11 +42,12 @@ EXPORTED_SYMBOLS = (
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
-    "cqa_set_key_prefetch",
+    "cqa_set_key_prefetch", "cqa_device_status",
 )
 
 PHASES = ("append_seal", "append_tail", "score", "select", "promote", "decide", "dense_keys",
-          "attend", "combine", "dense_attend", "dense_combine", "prefetch")
+          "attend", "combine", "dense_attend", "dense_combine", "prefetch", "naive",
+          "naive_combine")
 
 
 class _Config(ctypes.Structure):
@@ -129,12 +130,13 @@ def load_library() -> ctypes.CDLL:
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.cqa_dense_attention_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.cqa_set_key_prefetch.argtypes = [vp, i32, ctypes.c_float]
+    lib.cqa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
                  "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
                  "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
-                 "cqa_set_key_prefetch"):
+                 "cqa_set_key_prefetch", "cqa_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -235,6 +237,13 @@ def cqa_set_key_prefetch(handle, mode: int = 1, min_fraction: float = 0.75):
                   "cqa_set_key_prefetch")
 
 
+def cqa_device_status(handle) -> int:
+    """Synchronise and return (then clear) the device status word; 0 = all kernels normal."""
+    out = ctypes.c_int32()
+    _check(load_library().cqa_device_status(handle, ctypes.byref(out)), "cqa_device_status")
+    return int(out.value)
+
+
 def cqa_dense_attention_noalloc(q, k, v, out, stream=None):
     """Exact attention over caller-held FP16 keys and values that allocates no
     device memory (for callers that cannot call cudaMalloc; see include/cqa.h).
@@ -277,6 +286,9 @@ class Cache:
 
     def __exit__(self, *exc):
         self.close()
+
+    def device_status(self) -> int:
+        return cqa_device_status(self.handle)
 
     def set_key_prefetch(self, mode: int = 1, min_fraction: float = 0.75):
         return cqa_set_key_prefetch(self.handle, mode, min_fraction)

@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcqa.so")
 
 SOURCES = ["cqa_api.cu", "k_append.cu", "k_score.cu", "k_select.cu", "k_attend.cu", "k_combine.cu",
-           "k_promote.cu", "cqa_noalloc.cu"]
+           "k_promote.cu", "k_naive.cu", "cqa_noalloc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -193,6 +193,7 @@ const char* cqa_error_string(int code) {
     case CQA_ERR_OOM: return "out of memory";
     case CQA_ERR_CAPACITY: return "size exceeds a fixed capacity (cache max_ctx or scratch size)";
     case CQA_ERR_EMPTY: return "decode on an empty layer";
+    case CQA_ERR_TIMEOUT: return "a bounded device wait gave up (see cqa_device_status)";
   }
   return "unknown error";
 }
@@ -261,6 +262,8 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   const size_t o_dn = take(hq_rows);
   const size_t o_po = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * d * 4);
   const size_t o_ps = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
+  const size_t o_err = take(sizeof(int));
+  const size_t o_px = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     cudaGetLastError();
@@ -289,6 +292,8 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->sc.dense = (uint8_t*)(bp + o_dn);
   cc->sc.part_o = (float*)(bp + o_po);
   cc->sc.part_s = (float*)(bp + o_ps);
+  cc->sc.err = (int*)(bp + o_err);
+  cc->sc.part_x = (float*)(bp + o_px);
   cc->sc.ls = ls;
   cc->sc.max_chunks = (int)max_chunks;
 
@@ -482,6 +487,19 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   }
   const __half* kstage = slot >= 0 ? cc->kstage[slot] : nullptr;
   const int stage_nb = slot >= 0 ? cc->stage_nb[slot] : 0;
+  if (naive) {
+    // certification off: one streaming pass over Tier 1 and its combine
+    cudaError_t e = run_phase(cc, CQA_PHASE_NAIVE, s, 1, [&] {
+      return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung, 0, s);
+    });
+    if (e == cudaSuccess)
+      e = run_phase(cc, CQA_PHASE_NAIVE_COMBINE, s, 1, [&] {
+        return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung, 1, s);
+      });
+    if (e != cudaSuccess) return CQA_ERR_CUDA;
+    if (trace) return copy_trace(cc, sh, trace, s);
+    return CQA_OK;
+  }
   cudaError_t e = run_phase(cc, CQA_PHASE_SCORE, s, 1,
                             [&] { return launch_score(cc->t, cc->st, unit0, sh, qh, cc->sc, s); });
   if (e == cudaSuccess)
@@ -589,6 +607,19 @@ int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t b
     }
   }
   return (int64_t)total;
+}
+
+int cqa_device_status(cqa_cache* cc, int32_t* status) {
+  if (!cc || !status) return CQA_ERR_INVALID_ARG;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return CQA_ERR_CUDA;
+  if (cudaMemcpy(&v, cc->sc.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return CQA_ERR_CUDA;
+  if (v && cudaMemset(cc->sc.err, 0, sizeof(int)) != cudaSuccess) return CQA_ERR_CUDA;
+  *status = v;
+  return CQA_OK;
 }
 
 int cqa_set_key_prefetch(cqa_cache* cc, int mode, float min_fraction) {

@@ -83,6 +83,8 @@ struct Scratch {
   float* part_o;     // [B*Hkv][max_chunks][G][d]
   float* part_s;     // [B*Hkv][max_chunks][G][3]  (m, l, eta mass)
   int32_t* promo;    // [n_layers * B * Hkv] promoted block count per unit (pinned host, mapped)
+  int* err;          // device error word (bit 0: a bounded wait gave up)
+  float* part_x;     // [B*Hkv][max_chunks][G][3]  naive pass: (max Delta, residual m, residual l)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
 };
@@ -118,6 +120,10 @@ cudaError_t launch_select(const Tier1& t, const Strides& st, int layer_unit0,
 cudaError_t launch_attend(const Tier1& t, const Strides& st, int layer_unit0,
                           const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
                           cudaStream_t s);
+// certification off: part 0 = the streaming pass over Tier 1, part 1 = its combine
+cudaError_t launch_naive(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
+                         const __half* q, const Scratch& sc, float* out, float* e_key,
+                         float* e_val, uint8_t* rung, int part, cudaStream_t s);
 cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                            float* out, float* e_key, float* e_val, uint8_t* rung,
                            cudaStream_t s);

@@ -68,6 +68,7 @@ struct AttendSmem {
     float red[THREADS / LPR][D];
   } u;
   float m[G], l[G], e[G], alpha[G];
+  float eta_b;  // eta of the block being processed
 };
 
 // MODE 0: certified.  Logits come from scratch: INT8 for tail blocks, exact
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
     const size_t tok0 = resid ? (size_t)sh.nb * BLK : (size_t)j * BLK;  // token index
 
     // ---- logits ----
+    if (MODE == 0 && tid == 0 && !resid) S.eta_b = t.eta[u * st.eta + j];  // overlaps the loads below
     if (MODE == 0) {
       const float* lp = sc.logits + hrow0 * sc.ls + tok0;
       for (int e = tid; e < G * BLK; e += THREADS) {
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         S.l[h] = S.l[h] * alpha + lb;
         float ea = S.e[h] * alpha;
         const bool int4_here = MODE == 0 && !vprom && !sc.dense[hrow0 + h];
-        if (int4_here) ea += t.eta[u * st.eta + j] * lb;
+        if (int4_here) ea += S.eta_b * lb;
         S.e[h] = ea;
         S.m[h] = mnew;
         S.alpha[h] = alpha;

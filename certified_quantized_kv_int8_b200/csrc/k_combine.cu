@@ -104,55 +104,75 @@ __device__ __forceinline__ float cwarp_sum(float x) {
   return x;
 }
 
-// Merge the split-K partials of one head (a warp): returns o / L in o, and L, E.
+// Merge the split-K partials of one head with a CTA of D threads: thread c
+// returns channel c of o / L; every thread gets L and E.
 template <int D, int G>
-__device__ __forceinline__ void merge_head(const Scratch& sc, int nchunks, int unit, int hh,
-                                           int lane, float (&o)[D / 32], float& L, float& E) {
-  constexpr int CPL = D / 32;
+__device__ __forceinline__ float merge_head(const Scratch& sc, int nchunks, int unit, int hh,
+                                            float& L, float& E) {
+  constexpr int NW = D / 32;
+  __shared__ float wbuf[1024];
+  __shared__ float red[2][NW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = (size_t)unit * sc.max_chunks * G + hh;  // partial index of chunk 0
   float ml = -INFINITY;
-  for (int c = lane; c < nchunks; c += 32) ml = fmaxf(ml, sc.part_s[(base + (size_t)c * G) * 3]);
-  const float M = cwarp_max(ml);
+  for (int c = tid; c < nchunks; c += D) ml = fmaxf(ml, sc.part_s[(base + (size_t)c * G) * 3]);
+  ml = cwarp_max(ml);
+  if (lane == 0) red[0][warp] = ml;
+  __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, red[0][w]);
+  __syncthreads();
   float ll = 0.f, el = 0.f;
-  for (int c = lane; c < nchunks; c += 32) {
+  for (int c = tid; c < nchunks; c += D) {
     const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
     const float w = ps[0] == -INFINITY ? 0.f : expf(ps[0] - M);
+    if (c < 1024) wbuf[c] = w;
     ll += ps[1] * w;
     el += ps[2] * w;
   }
-  L = cwarp_sum(ll);
-  E = cwarp_sum(el);
+  ll = cwarp_sum(ll);
+  el = cwarp_sum(el);
+  if (lane == 0) {
+    red[0][warp] = ll;
+    red[1][warp] = el;
+  }
+  __syncthreads();
+  L = 0.f;
+  E = 0.f;
 #pragma unroll
-  for (int k = 0; k < CPL; ++k) o[k] = 0.f;
-#pragma unroll 4
+  for (int w = 0; w < NW; ++w) {
+    L += red[0][w];
+    E += red[1][w];
+  }
+  float o = 0.f;
+#pragma unroll 8
   for (int c = 0; c < nchunks; ++c) {
     const size_t pi = base + (size_t)c * G;
-    const float mc = sc.part_s[pi * 3];
-    const float w = mc == -INFINITY ? 0.f : expf(mc - M);
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) o[k] += sc.part_o[pi * D + lane + 32 * k] * w;
+    float w;
+    if (c < 1024) {
+      w = wbuf[c];
+    } else {
+      const float mc = sc.part_s[pi * 3];
+      w = mc == -INFINITY ? 0.f : expf(mc - M);
+    }
+    o = fmaf(sc.part_o[pi * D + tid], w, o);
   }
-  const float inv = 1.f / L;
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) o[k] *= inv;
+  return o / L;
 }
 
-// Outputs, E_val and the E_val post-check; one warp per (batch row, head).
+// Outputs, E_val and the E_val post-check; one CTA of D threads per (batch row, head).
 template <int D, int G>
 __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
                                float* __restrict__ out, float* __restrict__ e_key,
                                float* __restrict__ e_val, uint8_t* __restrict__ rung) {
-  constexpr int CPL = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // b * Hq + h
-  if (row >= sh.B * sh.Hq) return;
+  const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   const int g = h / G, hh = h - g * G;
-  float o[CPL], L, E;
-  merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, lane, o, L, E);
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) out[(size_t)row * D + lane + 32 * k] = o[k];
-  if (lane != 0) return;
+  float L, E;
+  const float o = merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, L, E);
+  out[(size_t)row * D + threadIdx.x] = o;
+  if (threadIdx.x != 0) return;
   const uint8_t dv = sc.dense[row];
   uint8_t hf = sc.hflags[row];
   const float ev = E / L;
@@ -175,23 +195,20 @@ __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
   sc.hflags[row] = hf;
 }
 
-// One warp per (batch row, query head): heads recomputed by a dense pass
-// (all heads for cqa_dense_reference, DENSE_LATE heads otherwise).
+// One CTA of D threads per (batch row, query head): heads recomputed by a
+// dense pass (all heads for cqa_dense_reference, DENSE_LATE heads otherwise).
 template <int D, int G>
 __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
                                      float* __restrict__ out, float* __restrict__ e_key,
                                      float* __restrict__ e_val, uint8_t* __restrict__ rung) {
-  constexpr int CPL = D / 32;
   const int row = blockIdx.x;  // b * Hq + h
-  const int lane = threadIdx.x;
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   if (!all_heads && !(sc.dense[row] & DENSE_LATE)) return;
   const int g = h / G, hh = h - g * G;
-  float o[CPL], L, E;
-  merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, lane, o, L, E);
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) out[(size_t)row * D + lane + 32 * k] = o[k];
-  if (!all_heads && lane == 0) {
+  float L, E;
+  const float o = merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, L, E);
+  out[(size_t)row * D + threadIdx.x] = o;
+  if (!all_heads && threadIdx.x == 0) {
     e_key[row] = 0.f;
     e_val[row] = 0.f;
     rung[row] = 3;
@@ -201,16 +218,15 @@ __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
 template <int D, int G>
 cudaError_t combine_t(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                       float* out, float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  const int rows = sh.B * sh.Hq;
-  combine_kernel<D, G><<<(rows + 7) / 8, 256, 0, s>>>(sh, th, sc, out, e_key, e_val, rung);
+  combine_kernel<D, G><<<sh.B * sh.Hq, D, 0, s>>>(sh, th, sc, out, e_key, e_val, rung);
   return cudaGetLastError();
 }
 
 template <int D, int G>
 cudaError_t dense_combine_t(const DecodeShape& sh, const Scratch& sc, int all_heads, float* out,
                             float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  dense_combine_kernel<D, G><<<sh.B * sh.Hq, 32, 0, s>>>(sh, sc, all_heads, out, e_key, e_val,
-                                                         rung);
+  dense_combine_kernel<D, G><<<sh.B * sh.Hq, D, 0, s>>>(sh, sc, all_heads, out, e_key, e_val,
+                                                        rung);
   return cudaGetLastError();
 }
 

@@ -51,7 +51,8 @@ enum {
   CQA_ERR_CUDA = -2,        /* a CUDA runtime call failed */
   CQA_ERR_OOM = -3,         /* device or pinned-host allocation failed */
   CQA_ERR_CAPACITY = -4,    /* an append beyond max_ctx, or a shape beyond a fixed scratch size */
-  CQA_ERR_EMPTY = -5        /* decode on a layer that holds no token */
+  CQA_ERR_EMPTY = -5,       /* decode on a layer that holds no token */
+  CQA_ERR_TIMEOUT = -6      /* reported by cqa_device_status: a device wait gave up */
 };
 
 typedef struct cqa_cache cqa_cache; /* opaque */
@@ -83,7 +84,7 @@ typedef struct cqa_thresholds {
   float layer_dense_frac; /* rung 4 when >= ceil(layer_dense_frac * n_q_heads) heads of a
                              (layer, batch row) took rung 3 */
   int32_t naive;          /* 1: certification off (no promotion, no ladder; bounds still
-                             reported), 0: certified */
+                             reported; one fused INT8/INT4 streaming pass), 0: certified */
 } cqa_thresholds;
 
 /* Optional per-call diagnostics, all device pointers, any may be NULL.
@@ -170,6 +171,13 @@ enum {
 };
 int64_t cqa_debug_export(cqa_cache* cache, int layer, int what, void* host_dst, size_t bytes);
 
+/* Device status word of the cache's kernels, read after synchronising the
+ * device and then cleared.  The streaming kernels wait for their own bulk
+ * copies with a bounded number of polls; a wait that runs out sets bit 0
+ * (and that kernel's results are not valid).  *status = 0 means every kernel
+ * since the last call completed normally. */
+int cqa_device_status(cqa_cache* cache, int32_t* status);
+
 /* Whole-layer key prefetch.  Promotion reads the FP16 keys of the selected
  * blocks from Tier 2.  When a layer's last decode promoted nearly all of its
  * blocks, copying the layer's sealed keys to device memory with the copy
@@ -203,7 +211,9 @@ enum {
   CQA_PHASE_DENSE_ATTEND = 9,  /* exact attention from Tier 2 (E_val post-check, reference) */
   CQA_PHASE_DENSE_COMBINE = 10,
   CQA_PHASE_PREFETCH = 11,     /* copy-engine copy of a layer's Tier-2 keys (not a kernel) */
-  CQA_PHASE_COUNT = 12
+  CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1 */
+  CQA_PHASE_NAIVE_COMBINE = 13,
+  CQA_PHASE_COUNT = 14
 };
 /* Start (or restart) profiling; max_launches bounds the recorded launches
  * (further launches are counted but not timed). */

@@ -187,6 +187,7 @@ def run_decode(cache, layer, q, th, stream=None):
     trace = cache.alloc_trace(layer)
     cache.decode(layer, q, th, outputs=outs, trace=trace, stream=stream)
     torch.cuda.synchronize()
+    assert cache.device_status() == 0, "a device wait gave up"
     res = dict(out=outs[0], e_key=outs[1], e_val=outs[2], rung=outs[3], **trace)
     return {k: v.cpu().numpy() for k, v in res.items()}
 

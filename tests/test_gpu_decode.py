@@ -189,3 +189,14 @@ def test_key_prefetch_changes_no_result(cqa):
         for a, b in zip(results[0], results[mode]):
             for x, y in zip(a, b):
                 assert np.array_equal(x, y), f"prefetch mode {mode} changed a result"
+
+
+@pytest.mark.parametrize("name,layer", [("llama8b_8k_1layer", 0), ("llama8b_64k_b4_t3values", 2),
+                                        ("llama8b_128k_needle", 17)])
+def test_naive_path_full_size(cqa, name, layer):
+    """Certification off: the fused INT8/INT4 streaming pass against the oracle's
+    naive mode (no promotion, bounds over the whole tail)."""
+    w = sk.WORKLOADS[name]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "naive": True})
+    log = _check(cqa, w, w.ctx + 33, th, layers=(layer,), label=f"naive {name}")
+    assert not log.entries
