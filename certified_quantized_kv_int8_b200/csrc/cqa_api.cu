@@ -4,7 +4,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "cqa_internal.cuh"
@@ -14,6 +17,22 @@ size_t select_smem_bytes(int G, int nb);
 }
 
 using namespace cqa;
+
+namespace cqa {
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> granted;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& g = granted[std::make_pair(kernel, dev)];
+  if (bytes <= g) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) g = bytes;
+  return e;
+}
+}  // namespace cqa
 
 struct cqa_cache {
   cqa_config cfg;

@@ -94,6 +94,11 @@ struct DecodeShape {
   float sigma;
 };
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
+// again only when a launch needs more than already granted: the attribute
+// call may stall the host, so it stays off the per-launch path.
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
+
 // ---- launchers (each returns the launch error, cudaSuccess on success) ----
 cudaError_t launch_seal(const Tier1& t, const Strides& st, int layer_unit0, int B, int Hkv, int d,
                         const __half* knew, const __half* vnew, int T_old, int n_new, int nb_old,

@@ -67,7 +67,9 @@ __device__ __forceinline__ void u4x8_f2(uint32_t w, float2 (&c)[4]) {
 template <int D, int G>
 struct NaiveSmem {
   float qf[G][D];        // q * sigma
-  float qs[G][D];        // q * sigma * key scale of the current block
+  float qs[G][D / 16][20];  // q * sigma * key scale of the current block; 16-channel rows
+                            // padded to 20 floats so the scoring warps' 16-byte reads
+                            // spread over all banks
   float lg[G][BLK];
   float pp[G][BLK];
   float red[NT / (D / 8)][D];
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
     // q * sigma * scale, and Delta_b per head (warp h)
     for (int e = tid; e < G * D; e += NT) {
       const int h = e / D, c = e - h * D;
-      S.qs[h][c] = S.qf[h][c] * ks[c];
+      S.qs[h][c >> 4][c & 15] = S.qf[h][c] * ks[c];
     }
     if (warp < G) {
       float a = 0.f;
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
       float2 qs2[G][8];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float4* qp = reinterpret_cast<const float4*>(&S.qs[h][cc * 16]);
+        const float4* qp = reinterpret_cast<const float4*>(&S.qs[h][cc][0]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float4 x = qp[i];
@@ -487,8 +489,7 @@ cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeSh
   naive_chunking(sh, sc.max_chunks, &cb, &nch);
   if (part == 0) {
     const int smem = NST * NaiveLayout<D>::STAGE;
-    cudaError_t e = cudaFuncSetAttribute(naive_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G>, (int)smem);
     if (e != cudaSuccess) return e;
     naive_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc,
                                                                       cb, nch);

@@ -302,8 +302,7 @@ cudaError_t launch_score_t(const Tier1& t, const Strides& st, int unit0, const D
   if (grid < need_res) grid = need_res;
   if (grid < 1) grid = 1;
   const int smem = WARPS * NSTAGE * stage_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(score_kernel<D, G>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G>, (int)smem);
   if (e != cudaSuccess) return e;
   score_kernel<D, G><<<grid, WARPS * 32, smem, s>>>(t, st, unit0, sh, q, sc, n_sealed, units);
   return cudaGetLastError();

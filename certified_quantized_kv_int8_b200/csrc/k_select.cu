@@ -288,8 +288,7 @@ cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const 
   int NP = 2;
   while (NP < sh.nb) NP <<= 1;
   const size_t smem = (size_t)G * NP * 8 + (size_t)G * sh.nb * 4 + 2 * (size_t)sh.nb;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_dynamic_smem((const void*)select_kernel<G>, (int)smem);
   if (e != cudaSuccess) return e;
   select_kernel<G><<<sh.B * sh.Hkv, THREADS, smem, s>>>(t, st, unit0, sh, th, sc, NP);
   return cudaGetLastError();
