@@ -409,6 +409,15 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
                                          "hbm": dp["hbm_bytes"]},
         "traffic": (rec["dram_bytes_per_block"] * census["blocks_per_layer"] if rec else None),
     }
+    # the host link over the whole certified step: key copies by the copy engine
+    # plus every kernel's host-link reads, against the pinned-copy rate
+    link_bytes = sum(p["host_link_bytes"] * p["launches"] for p in phases.values()) / args.steps
+    step_roofline = {
+        "bound": "h2d", "bytes_per_step": link_bytes,
+        "achieved": link_bytes / (t_max / args.steps) / 1e9, "peak": h2d_peak, "unit": "GB/s",
+        "peak_source": "pinned 1 GiB cudaMemcpyAsync H2D probe, this run",
+    }
+    step_roofline["frac"] = step_roofline["achieved"] / h2d_peak
     sp = phases["score"]
     rec_sc = traffic_record("score")
     roofline_hbm = {
@@ -447,6 +456,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         },
         "roofline": roofline,
         "roofline_hbm": roofline_hbm,
+        "step_roofline": step_roofline,
         "int8_int4_path": {
             "steps_per_s": n_naive * ws / n_max,
             "effective_kv_gbs": kv_gbs,

@@ -501,6 +501,9 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
     slot = staged_slot(cc, layer);
     if (slot >= 0 && cc->stage_nb[slot] != sh.nb) slot = -1;
     if (slot < 0 && want_prefetch(cc, layer)) slot = issue_prefetch(cc, layer, -1, s);
+    // the next layer's keys, copied while this layer runs: the copy shares the
+    // host link with this layer's value pass, which keeps the link busy through
+    // the scoring and selection phases that do not use it
     const int next = (layer + 1) % cc->cfg.n_layers;
     if (next != layer && want_prefetch(cc, next)) issue_prefetch(cc, next, slot, s);
   }

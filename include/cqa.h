@@ -183,9 +183,9 @@ int cqa_device_status(cqa_cache* cache, int32_t* status);
  * blocks, copying the layer's sealed keys to device memory with the copy
  * engine is faster than gathering them block by block, and the copy of the
  * next layer can run while the current layer computes.  With mode 1
- * (adaptive, the default) cqa_decode of layer l stages layer l and layer
- * (l + 1) % n_layers whenever their last decode promoted at least
- * min_fraction of their blocks (the first decode of a layer never does);
+ * (adaptive, the default) cqa_decode of layer l stages layer l (unless already
+ * staged) and layer (l + 1) % n_layers whenever their last decode promoted at
+ * least min_fraction of their blocks (the first decode of a layer never does);
  * mode 2 always stages; mode 0 never does.  Staging changes no result: the
  * promoted keys are the same bytes, and blocks the copy did not cover are
  * read from Tier 2 as before.  It uses two device buffers of one layer's
