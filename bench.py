@@ -291,12 +291,33 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     outs = cache.alloc_outputs()
     stream = torch.cuda.current_stream(device)
 
+    # the timed loops call the C entry points with marshalled arguments prepared
+    # once, so the host enqueues a layer in a few microseconds (the e2e pass below
+    # goes through the Python API instead)
+    import ctypes
+    lib = cqa.load_library()
+    c_stream = ctypes.c_void_p(stream.cuda_stream)
+    c_outs = [ctypes.c_void_p(t.data_ptr()) for t in outs]
+    c_th_keep = [th.as_c(), th_naive.as_c()]
+    c_th = {id(th): ctypes.byref(c_th_keep[0]), id(th_naive): ctypes.byref(c_th_keep[1])}
+    c_in = []
+    for qs_, kv_ in inputs:
+        c_in.append(([ctypes.c_void_p(x.data_ptr()) for x in qs_],
+                     [(ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr())) for k, v in kv_]))
+
     def run_step(s, thr):
-        qs, kv = inputs[s]
+        cq, ckv = c_in[s]
+        cth = c_th[id(thr)]
+        h = cache.handle
         for layer in range(L):
             if appends:
-                cache.append(layer, kv[layer][0], kv[layer][1], stream)
-            cache.decode(layer, qs[layer], thr, outputs=outs, stream=stream)
+                rc = lib.cqa_quantize_append(h, layer, ckv[layer][0], ckv[layer][1], 1, c_stream)
+                if rc:
+                    raise cqa.CqaError(rc, "cqa_quantize_append")
+            rc = lib.cqa_decode(h, layer, cq[layer], cth, c_outs[0], c_outs[1], c_outs[2],
+                                c_outs[3], None, c_stream)
+            if rc:
+                raise cqa.CqaError(rc, "cqa_decode")
 
     def timed(first, n, thr, profile=False, label="timed"):
         barrier(dist, device)

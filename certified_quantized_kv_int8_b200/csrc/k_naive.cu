@@ -20,7 +20,8 @@ namespace cqa {
 
 namespace {
 
-constexpr int NT = 256;  // threads per CTA
+constexpr int NT = 128;  // threads per CTA: four warps, four resident CTAs per SM
+constexpr int NW = NT / 32;
 constexpr int NST = 3;   // stages per CTA
 
 template <int D>
@@ -80,7 +81,7 @@ struct NaiveSmem {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int unit0,
+__global__ void __launch_bounds__(NT, 4) naive_kernel(Tier1 t, Strides st, int unit0,
                                                       DecodeShape sh,
                                                       const __half* __restrict__ q, Scratch sc,
                                                       int chunk_blocks, int nres_chunk) {
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
   constexpr int RPC = NT / LPR;
   constexpr int NPASS = BLK / RPC;
   constexpr int NG = D / VG;
-  constexpr int ROWS_PER_WARP = BLK / (NT / 32);  // 8 rows of a block per warp
+  constexpr int ROWS_PER_WARP = BLK / NW;  // 16 rows of a block per warp
   constexpr int NLW = ROWS_PER_WARP / RPW;
   static_assert(NLW >= 1, "layout");
 
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
       }
     }
     __syncthreads();
-    if (warp < G) softmax_step(warp, sh.r, &sc.ell_res[hrow0 + warp], 0.f, true);
+    for (int h = warp; h < G; h += NW) softmax_step(h, sh.r, &sc.ell_res[hrow0 + h], 0.f, true);
     __syncthreads();
     pv_rescale();
 #pragma unroll
@@ -269,14 +270,14 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
       const int h = e / D, c = e - h * D;
       S.qs[h][c >> 4][c & 15] = S.qf[h][c] * ks[c];
     }
-    if (warp < G) {
+    for (int h = warp; h < G; h += NW) {
       float a = 0.f;
-      for (int c = lane; c < D; c += 32) a = fmaf(fabsf(S.qf[warp][c]), ks[c], a);
+      for (int c = lane; c < D; c += 32) a = fmaf(fabsf(S.qf[h][c]), ks[c], a);
       a = nwarp_sum(a);
       if (lane == 0) {
         const float dl = 0.5f * a;
-        S.dmax[warp] = fmaxf(S.dmax[warp], dl);
-        sc.delta[(hrow0 + warp) * sh.nbm + j] = dl;
+        S.dmax[h] = fmaxf(S.dmax[h], dl);
+        sc.delta[(hrow0 + h) * sh.nbm + j] = dl;
       }
     }
     __syncthreads();
@@ -316,9 +317,8 @@ __global__ void __launch_bounds__(NT, 2) naive_kernel(Tier1 t, Strides st, int u
       }
     }
     __syncthreads();
-    if (warp < G) {
-      softmax_step(warp, BLK, &sc.ell8[(hrow0 + warp) * sh.nbm + j], S.eta[stg], false);
-    }
+    for (int h = warp; h < G; h += NW)
+      softmax_step(h, BLK, &sc.ell8[(hrow0 + h) * sh.nbm + j], S.eta[stg], false);
     if (tid == 0) sc.bflags[(size_t)unit * sh.nbm + j] = 0;  // nothing promoted
     __syncthreads();
 
@@ -468,10 +468,10 @@ __global__ void naive_combine_kernel(DecodeShape sh, Scratch sc, int nchunks, in
   }
 }
 
-// chunking of the streaming pass: about two resident CTAs per SM over all units
+// chunking of the streaming pass: about four resident CTAs per SM over all units
 void naive_chunking(const DecodeShape& sh, int max_chunks, int* cb, int* nch) {
   const int units = sh.B * sh.Hkv;
-  int per_unit = (148 * 2 + units - 1) / units;
+  int per_unit = (148 * 4 + units - 1) / units;
   if (per_unit > max_chunks - 1) per_unit = max_chunks - 1;  // one partial slot for the residual
   if (per_unit < 1) per_unit = 1;
   int c = sh.nb > 0 ? (sh.nb + per_unit - 1) / per_unit : 1;

@@ -200,3 +200,18 @@ def test_naive_path_full_size(cqa, name, layer):
     th = cqa.Thresholds(**{**sk.default_thresholds(w), "naive": True})
     log = _check(cqa, w, w.ctx + 33, th, layers=(layer,), label=f"naive {name}")
     assert not log.entries
+
+
+@pytest.mark.parametrize("d,hq,hkv", [(128, 8, 8), (128, 8, 4), (128, 16, 2), (64, 2, 2),
+                                      (64, 8, 2)])
+@pytest.mark.parametrize("naive", [False, True])
+def test_head_shapes(cqa, d, hq, hkv, naive):
+    """Every supported (head_dim, query heads per kv head) pair against the oracle,
+    with a tail (tau 0.8), value promotion and a batch of two."""
+    base = sk.WORKLOADS["tiny"]
+    w = dataclasses.replace(base, name=f"shape{d}_{hq}_{hkv}", batch=2, n_q_heads=hq,
+                            n_kv_heads=hkv, head_dim=d, n_outlier=2)
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.8, "v_tol": 3e-3,
+                           "naive": naive})
+    log = _check(cqa, w, 20 * 64 + 11, th, label=f"d{d} g{hq // hkv}")
+    assert len(log.entries) <= 1
