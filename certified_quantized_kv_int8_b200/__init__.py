@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
     "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
-    "cqa_set_key_prefetch", "cqa_device_status",
+    "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait",
 )
 
 PHASES = ("append_seal", "append_tail", "score", "select", "promote", "decide", "dense_keys",
@@ -131,12 +131,13 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_dense_attention_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
     lib.cqa_set_key_prefetch.argtypes = [vp, i32, ctypes.c_float]
     lib.cqa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.cqa_selftest_bounded_wait.argtypes = [vp, ctypes.c_int32]
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
                  "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
                  "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
-                 "cqa_set_key_prefetch", "cqa_device_status"):
+                 "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -242,6 +243,12 @@ def cqa_device_status(handle) -> int:
     out = ctypes.c_int32()
     _check(load_library().cqa_device_status(handle, ctypes.byref(out)), "cqa_device_status")
     return int(out.value)
+
+
+def cqa_selftest_bounded_wait(handle, polls: int = 1000):
+    """Launch a kernel whose bounded wait must give up (see include/cqa.h)."""
+    return _check(load_library().cqa_selftest_bounded_wait(handle, int(polls)),
+                  "cqa_selftest_bounded_wait")
 
 
 def cqa_dense_attention_noalloc(q, k, v, out, stream=None):

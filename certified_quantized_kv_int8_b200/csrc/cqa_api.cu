@@ -10,6 +10,7 @@
 #include <utility>
 #include <vector>
 
+#include "bulk_pipe.cuh"
 #include "cqa_internal.cuh"
 
 namespace cqa {
@@ -108,6 +109,18 @@ DecodeShape shape_of(const cqa_cache* c, int T) {
   sh.sigma = (float)(1.0 / sqrt((double)sh.d));
   chunking(sh.B * sh.Hkv, sh.nb, &sh.chunk_blocks, &sh.nchunks);
   return sh;
+}
+
+// A barrier nobody arrives on, waited for with a bounded number of polls: the
+// wait must give up and record ERR_TIMEOUT instead of hanging.
+__global__ void bounded_wait_selftest_kernel(int* err, uint32_t polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, err, polls);
 }
 
 __global__ void fill_range_kernel(float* vr, size_t units, int d) {
@@ -642,6 +655,14 @@ int cqa_device_status(cqa_cache* cc, int32_t* status) {
   if (v && cudaMemset(cc->sc.err, 0, sizeof(int)) != cudaSuccess) return CQA_ERR_CUDA;
   *status = v;
   return CQA_OK;
+}
+
+int cqa_selftest_bounded_wait(cqa_cache* cc, int32_t polls) {
+  if (!cc || polls < 1) return CQA_ERR_INVALID_ARG;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  bounded_wait_selftest_kernel<<<1, 32>>>(cc->sc.err, (uint32_t)polls);
+  return cudaGetLastError() == cudaSuccess ? CQA_OK : CQA_ERR_CUDA;
 }
 
 int cqa_set_key_prefetch(cqa_cache* cc, int mode, float min_fraction) {

@@ -145,18 +145,29 @@ __device__ __forceinline__ float merge_head(const Scratch& sc, int nchunks, int 
     L += red[0][w];
     E += red[1][w];
   }
+  // o: batches of 16 independent loads so the chain of chunk partials does not
+  // serialise on memory latency
   float o = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < nchunks; ++c) {
-    const size_t pi = base + (size_t)c * G;
-    float w;
-    if (c < 1024) {
-      w = wbuf[c];
-    } else {
-      const float mc = sc.part_s[pi * 3];
-      w = mc == -INFINITY ? 0.f : expf(mc - M);
+  for (int c0 = 0; c0 < nchunks; c0 += 16) {
+    float v[16], wv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = c0 + i;
+      v[i] = 0.f;
+      wv[i] = 0.f;
+      if (c < nchunks) {
+        const size_t pi = base + (size_t)c * G;
+        v[i] = sc.part_o[pi * D + tid];
+        if (c < 1024) {
+          wv[i] = wbuf[c];
+        } else {
+          const float mc = sc.part_s[pi * 3];
+          wv[i] = mc == -INFINITY ? 0.f : expf(mc - M);
+        }
+      }
     }
-    o = fmaf(sc.part_o[pi * D + tid], w, o);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o = fmaf(v[i], wv[i], o);
   }
   return o / L;
 }

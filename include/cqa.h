@@ -178,6 +178,12 @@ int64_t cqa_debug_export(cqa_cache* cache, int layer, int what, void* host_dst, 
  * since the last call completed normally. */
 int cqa_device_status(cqa_cache* cache, int32_t* status);
 
+/* Self-test of the failure path above: launches one kernel that waits, for at
+ * most `polls` polls, on a barrier nobody completes.  The wait gives up and
+ * sets bit 0 of the status word, which the next cqa_device_status returns;
+ * nothing faults or hangs.  Runs on the legacy default stream. */
+int cqa_selftest_bounded_wait(cqa_cache* cache, int32_t polls);
+
 /* Whole-layer key prefetch.  Promotion reads the FP16 keys of the selected
  * blocks from Tier 2.  When a layer's last decode promoted nearly all of its
  * blocks, copying the layer's sealed keys to device memory with the copy

@@ -102,3 +102,29 @@ def test_append_errors(cqa):
         cqa.Cache(1, 1, 6, 4, 64, 128)  # 6 query heads over 4 kv heads
     with pytest.raises(cqa.CqaError):
         cqa.Cache(1, 1, 4, 2, 96, 128)  # unsupported head_dim
+
+
+def test_bounded_wait_reports_instead_of_hanging(cqa):
+    """Failure detection without a fault: a device wait that nothing completes
+    gives up after its poll limit and the status word says so."""
+    with cqa.Cache(1, 1, 4, 2, 64, 128) as cache:
+        assert cache.device_status() == 0
+        cqa.cqa_selftest_bounded_wait(cache.handle, 2000)
+        assert cache.device_status() == 1  # read and cleared
+        assert cache.device_status() == 0
+        # the context stays usable
+        w = sk.WORKLOADS["tiny"]
+        K, V = sk.kv_layer(w, 0, 0, 100, "cuda")
+        cache.append(0, K, V)
+        out = cache.decode(0, sk.queries(w, 0, 0, "cuda"), cqa.Thresholds())[0]
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all()
+
+
+def test_allocation_failure_is_reported(cqa):
+    """A cache far larger than the device reports CQA_ERR_OOM and leaves nothing behind."""
+    with pytest.raises(cqa.CqaError) as e:
+        cqa.Cache(4096, 64, 32, 8, 128, 8192)  # ~2 TB of Tier 1
+    assert e.value.code == -3
+    with cqa.Cache(1, 1, 4, 2, 64, 128) as cache:  # the device still works
+        assert cache.device_status() == 0
