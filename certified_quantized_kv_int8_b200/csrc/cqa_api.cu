@@ -296,6 +296,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   const size_t o_ps = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
   const size_t o_err = take(sizeof(int));
   const size_t o_px = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
+  const size_t o_cnt = take((size_t)c.batch * c.n_kv_heads * sizeof(int));
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     cudaGetLastError();
@@ -326,6 +327,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->sc.part_s = (float*)(bp + o_ps);
   cc->sc.err = (int*)(bp + o_err);
   cc->sc.part_x = (float*)(bp + o_px);
+  cc->sc.cnt = (int*)(bp + o_cnt);
   cc->sc.ls = ls;
   cc->sc.max_chunks = (int)max_chunks;
 
@@ -523,14 +525,11 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   const __half* kstage = slot >= 0 ? cc->kstage[slot] : nullptr;
   const int stage_nb = slot >= 0 ? cc->stage_nb[slot] : 0;
   if (naive) {
-    // certification off: one streaming pass over Tier 1 and its combine
+    // certification off: one streaming pass over Tier 1 (its last CTA per unit combines)
     cudaError_t e = run_phase(cc, CQA_PHASE_NAIVE, s, 1, [&] {
-      return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung, 0, s);
+      return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung,
+                          trace != nullptr, s);
     });
-    if (e == cudaSuccess)
-      e = run_phase(cc, CQA_PHASE_NAIVE_COMBINE, s, 1, [&] {
-        return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung, 1, s);
-      });
     if (e != cudaSuccess) return CQA_ERR_CUDA;
     if (trace) return copy_trace(cc, sh, trace, s);
     return CQA_OK;
@@ -635,7 +634,13 @@ int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t b
       char* dp = out + (uu * parts + p) * per_unit;
       if (per_unit == 0) continue;
       if (host_src) {
-        memcpy(dp, sp, per_unit);
+        // sealed tokens from Tier 2; the residual block's from device memory
+        const size_t sealed = (size_t)nb * BLK * d * 2;
+        memcpy(dp, sp, sealed);
+        const char* rs = (const char*)(p == 0 ? cc->t.kres : cc->t.vres) + (unit0 + uu) * st.res * 2;
+        if (per_unit > sealed &&
+            cudaMemcpy(dp + sealed, rs, per_unit - sealed, cudaMemcpyDeviceToHost) != cudaSuccess)
+          return CQA_ERR_CUDA;
       } else if (cudaMemcpy(dp, sp, per_unit, cudaMemcpyDeviceToHost) != cudaSuccess) {
         return CQA_ERR_CUDA;
       }

@@ -85,6 +85,7 @@ struct Scratch {
   int32_t* promo;    // [n_layers * B * Hkv] promoted block count per unit (pinned host, mapped)
   int* err;          // device error word (bit 0: a bounded wait gave up)
   float* part_x;     // [B*Hkv][max_chunks][G][3]  naive pass: (max Delta, residual m, residual l)
+  int* cnt;          // [B*Hkv] naive pass: CTAs of the unit that have finished (0 between calls)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
 };
@@ -125,10 +126,12 @@ cudaError_t launch_select(const Tier1& t, const Strides& st, int layer_unit0,
 cudaError_t launch_attend(const Tier1& t, const Strides& st, int layer_unit0,
                           const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
                           cudaStream_t s);
-// certification off: part 0 = the streaming pass over Tier 1, part 1 = its combine
+// certification off: one streaming pass over Tier 1 whose last CTA per unit
+// merges the partials into the outputs; with `trace` set the pass also writes
+// the per-block ell8, Delta and block flags of the trace
 cudaError_t launch_naive(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
                          const __half* q, const Scratch& sc, float* out, float* e_key,
-                         float* e_val, uint8_t* rung, int part, cudaStream_t s);
+                         float* e_val, uint8_t* rung, int trace, cudaStream_t s);
 cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                            float* out, float* e_key, float* e_val, uint8_t* rung,
                            cudaStream_t s);

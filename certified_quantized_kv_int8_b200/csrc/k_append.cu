@@ -1,5 +1,8 @@
-// Append path: seal complete 64-token blocks into Tier 1, keep the residual
-// block exact, write every new token to Tier 2.
+// Append path: seal complete 64-token blocks into Tier 1 and copy them to
+// Tier 2; keep the residual (unsealed) block exact in device memory.  A token
+// reaches Tier 2 when its block seals: until then only the residual block,
+// never promoted, holds it, so appends of single tokens touch device memory
+// alone and the host link carries whole blocks.
 //
 // Runtime-Certified Bounded-Error Quantized Attention, Methodology §1
 // (tiered storage): Tier 1 holds per-channel INT8 keys and per-group INT4
@@ -69,6 +72,14 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
   if (threadIdx.x == 0) eta_bits = 0;
   __syncthreads();
 
+  // the block's FP16 originals to Tier 2 (pinned host memory, device-mapped)
+  for (int e = threadIdx.x; e < BLK * C8; e += blockDim.x) {
+    const int tk = e / C8, c8 = e % C8;
+    const size_t dst2 = u * st.tier2 + ((size_t)j * BLK + tk) * D + c8 * 8;
+    *reinterpret_cast<uint4*>(t.k2 + dst2) = reinterpret_cast<const uint4*>(ks)[e];
+    *reinterpret_cast<uint4*>(t.v2 + dst2) = reinterpret_cast<const uint4*>(vs)[e];
+  }
+
   // per-channel key scale
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float a = 0.f;
@@ -133,8 +144,8 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
   if (threadIdx.x == 0) t.eta[u * st.eta + j] = __int_as_float(eta_bits);
 }
 
-// grid (ceil(n_new/64), B*Hkv), 256 threads: Tier-2 copy, residual slots,
-// per-channel value range.
+// grid (ceil(n_new/64), B*Hkv), 256 threads: residual slots, per-channel
+// value range.
 template <int D>
 __global__ void __launch_bounds__(256) append_tail_kernel(Tier1 t, Strides st, int unit0,
                                                           const __half* __restrict__ knew,
@@ -149,12 +160,9 @@ __global__ void __launch_bounds__(256) append_tail_kernel(Tier1 t, Strides st, i
     const int i = i0 + e / C8, c8 = e % C8;
     const int tok = T_old + i;
     const size_t src = ((size_t)ug * n_new + i) * D + c8 * 8;
-    const uint4 kv = *reinterpret_cast<const uint4*>(knew + src);
-    const uint4 vv = *reinterpret_cast<const uint4*>(vnew + src);
-    const size_t dst2 = u * st.tier2 + (size_t)tok * D + c8 * 8;
-    *reinterpret_cast<uint4*>(t.k2 + dst2) = kv;
-    *reinterpret_cast<uint4*>(t.v2 + dst2) = vv;
     if (tok >= nb_new * BLK) {
+      const uint4 kv = *reinterpret_cast<const uint4*>(knew + src);
+      const uint4 vv = *reinterpret_cast<const uint4*>(vnew + src);
       const size_t dr = u * st.res + (size_t)(tok - nb_new * BLK) * D + c8 * 8;
       *reinterpret_cast<uint4*>(t.kres + dr) = kv;
       *reinterpret_cast<uint4*>(t.vres + dr) = vv;

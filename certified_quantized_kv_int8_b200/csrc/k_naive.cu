@@ -13,6 +13,29 @@
 // through a ring of NST shared-memory stages filled by bulk copies (INT8
 // codes, key scales, INT4 codes, value scale/offset of one block per stage):
 // 14.5 KiB per block for head_dim 128, every byte of Tier 1 read once.
+//
+// The pass is bound by instruction issue as much as by HBM (per token and kv
+// head: 128 INT8 and 128 INT4 conversions and 2*G*head_dim multiply-adds
+// against 232 bytes), so the layout is chosen to spend few instructions
+// besides those:
+//   * one CTA barrier per block: it publishes the block's scaled queries
+//     (double-buffered by block parity) and releases the previous block's
+//     stage to the copy engine;
+//   * each warp owns 16 tokens of every block and keeps its own online
+//     softmax state, so the softmax and the P.V step need only warp-level
+//     synchronisation; the four warps' states merge once per chunk;
+//   * logits: sixteen lanes per token, 8 channels each; the G partial dots are
+//     reduced with a reduce-scatter whose register order is permuted per lane
+//     (register r of a lane holds head r ^ pi(lane)), so no selects are needed
+//     and each level halves the values in flight;
+//   * logits are kept in base 2 (queries pre-scaled by log2 e) so every
+//     exponential is one exp2;
+//   * INT4 codes become floats by masking a nibble into the mantissa of 2^23
+//     (nibbles 0-4 of a word in place, 5-7 after one shift) and one packed
+//     subtraction; nibble k then carries a power-of-two factor 16^k that is
+//     divided out of its accumulator once per chunk (exact);
+//   * the value scale is folded into the attention weight per (token, group,
+//     head) by the softmax lanes, which also accumulate the offset term.
 #include "bulk_pipe.cuh"
 #include "cqa_internal.cuh"
 
@@ -20,9 +43,12 @@ namespace cqa {
 
 namespace {
 
-constexpr int NT = 128;  // threads per CTA: four warps, four resident CTAs per SM
+constexpr int NT = 128;  // threads per CTA: four warps
 constexpr int NW = NT / 32;
-constexpr int NST = 3;   // stages per CTA
+constexpr int NST = 3;         // stages per CTA
+constexpr int TPW = BLK / NW;  // tokens of each block handled by one warp
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
 
 template <int D>
 struct NaiveLayout {
@@ -31,6 +57,15 @@ struct NaiveLayout {
   static constexpr int VB = BLK * D / 2;          // INT4 value codes
   static constexpr int MB = BLK * (D / VG) * 8;   // value scale/offset
   static constexpr int STAGE = KB + SB + VB + MB;
+};
+
+// channels per lane in the logit step.  The lane holds its channels' scaled
+// queries for every head in registers; 8 channels (16 lanes per token) keep the
+// kernel within 128 registers with the P.V accumulators, where 16 channels
+// spill and issue fewer instructions per cycle, for the same count.
+template <int G>
+struct NaiveLanes {
+  static constexpr int CH = 8;
 };
 
 __device__ __forceinline__ float nwarp_max(float x) {
@@ -45,6 +80,8 @@ __device__ __forceinline__ float nwarp_sum(float x) {
   return x;
 }
 
+// four INT8 codes -> floats: bias to unsigned, place each byte in the
+// mantissa of 2^23, subtract 2^23 + 128 (exact)
 __device__ __forceinline__ void s8x4_f2(uint32_t w, float2& a, float2& b) {
   const uint32_t u = w ^ 0x80808080u;
   const float2 off = make_float2(-8388736.0f, -8388736.0f);
@@ -54,50 +91,231 @@ __device__ __forceinline__ void s8x4_f2(uint32_t w, float2& a, float2& b) {
                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653))), off);
 }
 
-__device__ __forceinline__ void u4x8_f2(uint32_t w, float2 (&c)[4]) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+// eight INT4 codes (nibble k = channel k) -> c[k/2] = (n_k * 16^e_k, n_k+1 * 16^e_k+1)
+// with e = 0,1,2,3,4,0,1,2
+__device__ __forceinline__ void u4x8_scaled(uint32_t w, float2 (&c)[4]) {
+  const uint32_t m = 0x4B000000u;
+  const uint32_t h = w >> 20;
   const float2 off = make_float2(-8388608.0f, -8388608.0f);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t sel = 0x7650u + (uint32_t)i;
-    c[i] = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, sel)),
-                                  __uint_as_float(__byte_perm(hi, 0x4B000000u, sel))), off);
-  }
+  c[0] = __fadd2_rn(make_float2(__uint_as_float((w & 0xFu) | m),
+                                __uint_as_float((w & 0xF0u) | m)), off);
+  c[1] = __fadd2_rn(make_float2(__uint_as_float((w & 0xF00u) | m),
+                                __uint_as_float((w & 0xF000u) | m)), off);
+  c[2] = __fadd2_rn(make_float2(__uint_as_float((w & 0xF0000u) | m),
+                                __uint_as_float((h & 0xFu) | m)), off);
+  c[3] = __fadd2_rn(make_float2(__uint_as_float((h & 0xF0u) | m),
+                                __uint_as_float((h & 0xF00u) | m)), off);
 }
 
+// 2^x by the hardware approximation (relative error about 2^-22; flushes
+// results below 2^-126 to zero, which only drops weights that small)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 16^-e of nibble k (see u4x8_scaled)
+__device__ __forceinline__ float nib_unscale(int k) {
+  const int e = k < 5 ? k : k - 5;
+  return __int_as_float((127 - 4 * e) << 23);
+}
+
+// float offsets in the stage area where the merge of a unit's partials starts:
+// after the residual CTA's logits and statistics, after the main CTAs' per-warp
+// states (multiples of 4 floats, so the merge's float4 scratch stays aligned)
 template <int D, int G>
-struct NaiveSmem {
-  float qf[G][D];        // q * sigma
-  float qs[G][D / 16][20];  // q * sigma * key scale of the current block; 16-channel rows
-                            // padded to 20 floats so the scoring warps' 16-byte reads
-                            // spread over all banks
-  float lg[G][BLK];
-  float pp[G][BLK];
-  float red[NT / (D / 8)][D];
-  float m[G], l[G], e[G], alpha[G], dmax[G];
-  float mres[G], lres[G];
-  float eta[NST];  // eta_b of the block held by each stage
-  uint64_t bar[NST];
+struct NaiveMergeAt {
+  static constexpr int RES = (G * BLK + 2 * G + 3) / 4 * 4;
+  static constexpr int MAIN = NW * G * (D + D / VG + 3);
+  static constexpr int AT = RES > MAIN ? RES : MAIN;
+  static_assert(MAIN % 4 == 0, "alignment");
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(NT, 4) naive_kernel(Tier1 t, Strides st, int unit0,
-                                                      DecodeShape sh,
-                                                      const __half* __restrict__ q, Scratch sc,
-                                                      int chunk_blocks, int nres_chunk) {
+struct NaiveSmem {
+  static constexpr int CH = NaiveLanes<G>::CH;
+  float qf[G][D];                  // q * sigma * log2(e)
+  float qs[2][G][D / CH][CH + 4];  // qf * key scale of the block, by block parity; rows padded
+                                   // by 4 floats so eight lanes' 16-byte reads hit distinct banks
+  float ws[NW][TPW][D / VG][G];    // attention weight * value scale per (token, group, head)
+  float alpha[NW][G];              // rescale factor of each warp's running state
+  float ellp[2][NW][G];            // trace: log2-sum-exp of each warp's tokens of a block
+  float dmax[G];
+  float eta[NST];  // eta_b of the block held by each stage
+  int last;        // this CTA merges its unit's partials
+  uint64_t bar[NST];
+};
+
+__device__ double naive_e_key(double dT, double dA, double m8T) {
+  const double a = m8T * exp(dT);
+  const double m_ub = a > 0.0 ? a / (a + (1.0 - m8T) * exp(-dA)) : 0.0;
+  return fmin(tanh(0.5 * dT), m_ub * expm1(2.0 * dT));
+}
+
+// Arrival of one CTA of a (batch row, kv head) unit; the last of its nparts
+// CTAs merges the unit's partials (split-K combine) into the outputs: the
+// outputs o / L, E_key from the largest Delta and the residual's mass, and
+// E_val = sum of eta-weighted mass / L.  Every CTA of the launch calls this
+// exactly once, also after a failed wait, so the arrival counter returns to
+// zero for the next launch.
+template <int D, int G>
+__device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int nparts, int unit,
+                                   size_t hrow0, float* __restrict__ out,
+                                   float* __restrict__ e_key, float* __restrict__ e_val,
+                                   uint8_t* __restrict__ rung, float* wsm, int* flag) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __threadfence();  // this thread's partials, before the arrival below
+  __syncthreads();
+  if (tid == 0) *flag = atomicAdd(&sc.cnt[unit], 1) == nparts - 1;
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  const size_t base = (size_t)unit * sc.max_chunks * G;  // partial index of (chunk 0, head 0)
+  float* wt = wsm;                  // [nparts][G] weights exp(m_c - M)
+  float* hs = wsm + nparts * G;     // [G] 1 / L
+  // per head (one warp each): the parts' (m, l, e, max Delta) are loaded in one
+  // round when they fit a lane's registers (up to 32 * PPL parts), else twice
+  constexpr int PPL = 4;  // parts per lane per round
+  for (int h = warp; h < G; h += NW) {
+    float M = -INFINITY, dA = 0.f, ll = 0.f, el = 0.f;
+    float mv[PPL], lv[PPL], ev[PPL];
+    for (int c0 = 0; c0 < nparts; c0 += 32 * PPL) {
+      float dv[PPL];
+#pragma unroll
+      for (int i = 0; i < PPL; ++i) {
+        const int c = c0 + i * 32 + lane;
+        const float* ps = sc.part_s + (base + (size_t)c * G + h) * 3;
+        const bool in = c < nparts;
+        mv[i] = in ? __ldcg(ps) : -INFINITY;
+        lv[i] = in ? __ldcg(ps + 1) : 0.f;
+        ev[i] = in ? __ldcg(ps + 2) : 0.f;
+        dv[i] = in ? __ldcg(&sc.part_x[(base + (size_t)c * G + h) * 3]) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < PPL; ++i) {
+        M = fmaxf(M, mv[i]);
+        dA = fmaxf(dA, dv[i]);
+      }
+    }
+    M = nwarp_max(M);
+    dA = nwarp_max(dA);
+    for (int c0 = 0; c0 < nparts; c0 += 32 * PPL) {
+      if (nparts > 32 * PPL) {  // the registers hold the last round only: reload
+#pragma unroll
+        for (int i = 0; i < PPL; ++i) {
+          const int c = c0 + i * 32 + lane;
+          const float* ps = sc.part_s + (base + (size_t)c * G + h) * 3;
+          const bool in = c < nparts;
+          mv[i] = in ? __ldcg(ps) : -INFINITY;
+          lv[i] = in ? __ldcg(ps + 1) : 0.f;
+          ev[i] = in ? __ldcg(ps + 2) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < PPL; ++i) {
+        const int c = c0 + i * 32 + lane;
+        const float w = mv[i] == -INFINITY ? 0.f : expf(mv[i] - M);
+        if (c < nparts) wt[c * G + h] = w;
+        ll = fmaf(lv[i], w, ll);
+        el = fmaf(ev[i], w, el);
+      }
+    }
+    const float L = nwarp_sum(ll), E = nwarp_sum(el);
+    if (lane == 0) {
+      const size_t row = hrow0 + h;
+      hs[h] = 1.f / L;
+      // the residual CTA (the last part) holds the residual's own statistics
+      const float* px = sc.part_x + (base + (size_t)(nparts - 1) * G + h) * 3;
+      const float mr = __ldcg(px + 1);
+      const double mres = mr == -INFINITY ? 0.0 : (double)__ldcg(px + 2) * exp((double)mr - M) / L;
+      const float ek = sh.nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
+      e_key[row] = ek;
+      e_val[row] = E / L;
+      rung[row] = 0;
+      sc.ekey[row] = ek;
+      sc.hflags[row] = 0;
+      sc.kstar[row] = 0;
+      sc.dense[row] = 0;
+    }
+  }
+  __syncthreads();
+  // outputs: float4 items (head, 4 channels); PS threads split the parts of an item
+  constexpr int NI = G * D / 4;
+  constexpr int PS = NI >= NT ? 1 : NT / NI;
+  float4* red = reinterpret_cast<float4*>(wsm + nparts * G + G + (4 - (nparts * G + G) % 4) % 4);
+  for (int it = tid; it < NI * PS; it += NT) {
+    const int item = it % NI, sl = it / NI;
+    const int h = item / (D / 4), c4 = item % (D / 4);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = sl; c0 < nparts; c0 += 16 * PS) {
+      float4 v[16];
+      float wv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = c0 + i * PS;
+        const bool in = c < nparts;
+        v[i] = in ? __ldcg(reinterpret_cast<const float4*>(
+                        sc.part_o + (base + (size_t)c * G + h) * D) + c4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        wv[i] = in ? wt[c * G + h] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        o.x = fmaf(v[i].x, wv[i], o.x);
+        o.y = fmaf(v[i].y, wv[i], o.y);
+        o.z = fmaf(v[i].z, wv[i], o.z);
+        o.w = fmaf(v[i].w, wv[i], o.w);
+      }
+    }
+    if (PS == 1) {
+      const float il = hs[h];
+      reinterpret_cast<float4*>(out + (hrow0 + h) * D)[c4] =
+          make_float4(o.x * il, o.y * il, o.z * il, o.w * il);
+    } else {
+      red[it] = o;
+    }
+  }
+  if (PS > 1) {
+    __syncthreads();
+    for (int item = tid; item < NI; item += NT) {
+      const int h = item / (D / 4), c4 = item % (D / 4);
+      float4 o = red[item];
+      for (int sl = 1; sl < PS; ++sl) {
+        const float4 t2 = red[sl * NI + item];
+        o.x += t2.x; o.y += t2.y; o.z += t2.z; o.w += t2.w;
+      }
+      const float il = hs[h];
+      reinterpret_cast<float4*>(out + (hrow0 + h) * D)[c4] =
+          make_float4(o.x * il, o.y * il, o.z * il, o.w * il);
+    }
+  }
+  if (tid == 0) sc.cnt[unit] = 0;  // every CTA of this launch has arrived
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
+    naive_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
+                 Scratch sc, int chunk_blocks, int nres_chunk, int trace,
+                 float* __restrict__ out, float* __restrict__ e_key, float* __restrict__ e_val,
+                 uint8_t* __restrict__ rung) {
   using LY = NaiveLayout<D>;
-  constexpr int CPT = D / 16;   // lanes per token row in the scoring step (16 channels each)
-  constexpr int RPW = 32 / CPT;
-  constexpr int LPR = D / 8;    // threads per token row in the P.V step (8 channels each)
-  constexpr int RPC = NT / LPR;
-  constexpr int NPASS = BLK / RPC;
   constexpr int NG = D / VG;
-  constexpr int ROWS_PER_WARP = BLK / NW;  // 16 rows of a block per warp
-  constexpr int NLW = ROWS_PER_WARP / RPW;
-  static_assert(NLW >= 1, "layout");
+  constexpr int CH = NaiveLanes<G>::CH;
+  constexpr int CPT = D / CH;        // lanes per token row in the logit step
+  constexpr int RPW = 32 / CPT;      // rows per warp instruction
+  constexpr int NLI = TPW / RPW;     // logit iterations per block
+  constexpr int LPT = D / 8;         // lanes per token row in the P.V step (8 channels each)
+  constexpr int TPI = 32 / LPT;
+  constexpr int NPI = TPW / TPI;
+  constexpr int NDUP = CPT > G ? CPT / G : 1;  // lanes holding the same (token, head) logit
+  constexpr int GPL = NG > NDUP ? NG / NDUP : 1;  // value groups per softmax lane
+  constexpr int QI = G * D / 4;                   // float4 items of the scaled queries
+  constexpr int NQI = (QI + NT - 1) / NT;
+  static_assert(NLI >= 1 && NPI >= 1 && RPW * NLI == TPW, "layout");
 
   extern __shared__ __align__(128) unsigned char dsm[];
-  __shared__ NaiveSmem<D, G> S;
+  __shared__ __align__(16) NaiveSmem<D, G> S;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.y;
@@ -105,24 +323,88 @@ __global__ void __launch_bounds__(NT, 4) naive_kernel(Tier1 t, Strides st, int u
   const size_t u = (size_t)unit0 + unit;
   const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
   const int chunk = blockIdx.x;
-  const int j0 = chunk * chunk_blocks;
-  const int j1 = chunk == nres_chunk ? j0 : min(sh.nb, j0 + chunk_blocks);
-  const int nblk = max(0, j1 - j0);
+  const size_t pbase = ((size_t)unit * sc.max_chunks + chunk) * G;
+  const float s2 = sh.sigma * LOG2E;
 
   for (int e = tid; e < G * D; e += NT) {
     const int h = e / D, c = e - h * D;
-    S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * sh.sigma;
+    S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * s2;
   }
-  if (tid < G) {
-    S.m[tid] = -INFINITY;
-    S.l[tid] = 0.f;
-    S.e[tid] = 0.f;
-    S.dmax[tid] = 0.f;
-    S.mres[tid] = -INFINITY;
-    S.lres[tid] = 0.f;
+  if (tid < G) S.dmax[tid] = 0.f;  // published by the barrier before the first block
+
+  // ---- the exact residual block: a CTA of its own (the last chunk index) ----
+  if (chunk == nres_chunk) {
+    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK] base-2 logits, then weights
+    float* mst = lg + G * BLK;                  // [G][2]
+    const int r = sh.r;
+    __syncthreads();
+    const __half* kr = t.kres + u * st.res;
+    const __half* vr = t.vres + u * st.res;
+    constexpr int CPL = D / 32;
+    for (int tt = warp; tt < r; tt += NW) {
+      float kf[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; i += 2) {
+        const float2 f = __half22float2(
+            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
+        kf[i] = f.x;
+        kf[i + 1] = f.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
+        v = nwarp_sum(v);
+        if (lane == 0) lg[h * BLK + tt] = v;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += NW) {
+      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
+      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
+      const float m = nwarp_max(fmaxf(x0, x1));
+      const float e0 = lane < r ? exp2f(x0 - m) : 0.f;
+      const float e1 = lane + 32 < r ? exp2f(x1 - m) : 0.f;
+      const float l = nwarp_sum(e0 + e1);
+      lg[h * BLK + lane] = e0;
+      lg[h * BLK + lane + 32] = e1;
+      if (lane == 0) {
+        mst[2 * h] = r > 0 ? m * LN2 : -INFINITY;
+        mst[2 * h + 1] = l;
+        sc.ell_res[hrow0 + h] = r > 0 ? (m + log2f(l)) * LN2 : -INFINITY;
+      }
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += NT) {
+      float o[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) o[h] = 0.f;
+      for (int tt = 0; tt < r; ++tt) {
+        const float v = __half2float(vr[(size_t)tt * D + c]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = fmaf(lg[h * BLK + tt], v, o[h]);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) sc.part_o[(pbase + h) * D + c] = o[h];
+    }
+    if (tid < G) {
+      sc.part_s[(pbase + tid) * 3 + 0] = mst[2 * tid];
+      sc.part_s[(pbase + tid) * 3 + 1] = mst[2 * tid + 1];
+      sc.part_s[(pbase + tid) * 3 + 2] = 0.f;
+      sc.part_x[(pbase + tid) * 3 + 0] = 0.f;
+      sc.part_x[(pbase + tid) * 3 + 1] = mst[2 * tid];
+      sc.part_x[(pbase + tid) * 3 + 2] = mst[2 * tid + 1];
+    }
+    naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
+                             reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::RES, &S.last);
+    return;
   }
+
+  const int j0 = chunk * chunk_blocks;
+  const int nblk = max(0, min(sh.nb, j0 + chunk_blocks) - j0);
   if (tid == 0) {
-    for (int s2 = 0; s2 < NST; ++s2) mbar_init(&S.bar[s2], 1);
+    for (int s = 0; s < NST; ++s) mbar_init(&S.bar[s], 1);
     mbar_init_fence();
   }
   __syncthreads();
@@ -143,340 +425,315 @@ __global__ void __launch_bounds__(NT, 4) naive_kernel(Tier1 t, Strides st, int u
   if (tid == 0)
     for (int k = 0; k < NST; ++k) issue(k);
 
-  const int row = tid / LPR, cl = tid - row * LPR;  // P.V layout
-  float2 acc[G][4];
-  float zacc[G];
+  // lane roles
+  const int cc = lane % CPT, tr = lane / CPT;  // logit step: channel slice, row
+  int pi = 0;                                  // head permutation of the reduce-scatter
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    zacc[h] = 0.f;
+  for (int m = CPT / 2, n = G; m >= 1; m >>= 1, n >>= 1)
+    if (n > 1 && (cc & m)) pi |= n / 2;
+  const int dup = cc & (NDUP - 1);
+  const bool owner = tr == 0 && dup == 0;  // one lane per head of the warp
+  const int cl = lane % LPT, ts = lane / LPT;  // P.V step: channel slice, row
+  const int gq = cl * 8 / VG;
+
+  float2 acc[G][4];  // P.V accumulators, channel 8*cl + k carries 16^e_k
+#pragma unroll
+  for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
-  }
+  float zl[GPL];  // offset term: sum of weight * value offset, per owned group of head pi
+#pragma unroll
+  for (int i = 0; i < GPL; ++i) zl[i] = 0.f;
+  float mrun = -INFINITY, lrun = 0.f, erun = 0.f;  // running state of head pi (base 2)
 
-  // online-softmax update of head h (warp h) from S.lg[h]; writes S.pp[h]
-  auto softmax_step = [&](int h, int ntok, float* ell_out, float eta_b, bool resid) {
-    const float x0 = lane < ntok ? S.lg[h][lane] : -INFINITY;
-    const float x1 = lane + 32 < ntok ? S.lg[h][lane + 32] : -INFINITY;
-    const float mb = nwarp_max(fmaxf(x0, x1));
-    const float e0 = expf(x0 - mb), e1 = expf(x1 - mb);
-    const float sb = nwarp_sum(e0 + e1);
-    const float mold = S.m[h];
-    const float mnew = fmaxf(mold, mb);
-    const float alpha = mold == -INFINITY ? 0.f : expf(mold - mnew);
-    const float c = expf(mb - mnew);
-    S.pp[h][lane] = e0 * c;
-    S.pp[h][lane + 32] = e1 * c;
-    if (lane == 0) {
-      const float lb = sb * c;
-      S.l[h] = S.l[h] * alpha + lb;
-      S.e[h] = S.e[h] * alpha + eta_b * lb;
-      S.m[h] = mnew;
-      S.alpha[h] = alpha;
-      if (ell_out) *ell_out = mb + logf(sb);
-      if (resid) {
-        S.mres[h] = mb;
-        S.lres[h] = sb;
-      }
-    }
-  };
-
-  auto pv_rescale = [&]() {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float al = S.alpha[h];
-      zacc[h] *= al;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[h][i].x *= al;
-        acc[h][i].y *= al;
-      }
-    }
-  };
-
-  // ---- the exact residual block: a CTA of its own (the last chunk index) ----
-  const bool res_cta = chunk == nres_chunk;
-  if (res_cta && sh.r > 0) {
-    const __half* kr = t.kres + u * st.res;
-    const __half* vr = t.vres + u * st.res;
-    // LPR threads per token row, 8 channels each; partial dots reduced over the row
-#pragma unroll
-    for (int p = 0; p < NPASS; ++p) {
-      const int tt = p * RPC + row;
-      float2 kf[4];
-      if (tt < sh.r) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(kr + (size_t)tt * D + cl * 8);
-        const __half2* kh = reinterpret_cast<const __half2*>(&kv);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) kf[i] = __half22float2(kh[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) kf[i] = make_float2(0.f, 0.f);
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v = fmaf(S.qf[h][cl * 8 + 2 * i], kf[i].x, v);
-          v = fmaf(S.qf[h][cl * 8 + 2 * i + 1], kf[i].y, v);
-        }
-#pragma unroll
-        for (int m = LPR / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-        if (cl == 0) S.lg[h][tt] = tt < sh.r ? v : -INFINITY;
-      }
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += NW) softmax_step(h, sh.r, &sc.ell_res[hrow0 + h], 0.f, true);
-    __syncthreads();
-    pv_rescale();
-#pragma unroll
-    for (int p = 0; p < NPASS; ++p) {
-      const int tt = p * RPC + row;
-      if (tt >= sh.r) continue;
-      const uint4 vv = *reinterpret_cast<const uint4*>(vr + (size_t)tt * D + cl * 8);
-      const __half2* vh = reinterpret_cast<const __half2*>(&vv);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 vf = __half22float2(vh[i]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float w = S.pp[h][tt];
-          acc[h][i] = __ffma2_rn(make_float2(w, w), vf, acc[h][i]);
-        }
-      }
-    }
-    __syncthreads();
-  } else if (res_cta && tid < G) {
-    sc.ell_res[hrow0 + tid] = -INFINITY;
-  }
-
-  // ---- the chunk's sealed blocks ----
   bool ok = true;
   int k = 0;
-  const int cc = lane % CPT, tr = lane / CPT;
   for (; k < nblk; ++k) {
     const int j = j0 + k;
     const int stg = k % NST;
-    ok = mbar_wait(&S.bar[stg], (uint32_t)((k / NST) & 1), sc.err);
-    if (!ok) break;
+    const bool got = mbar_wait(&S.bar[stg], (uint32_t)((k / NST) & 1), sc.err);
     const unsigned char* sp = dsm + (size_t)stg * LY::STAGE;
-    const uint4* kc = reinterpret_cast<const uint4*>(sp);
     const float* ks = reinterpret_cast<const float*>(sp + LY::KB);
     const uint8_t* vc = sp + LY::KB + LY::SB;
     const float* vm = reinterpret_cast<const float*>(sp + LY::KB + LY::SB + LY::VB);
 
-    // q * sigma * scale, and Delta_b per head (warp h)
-    for (int e = tid; e < G * D; e += NT) {
-      const int h = e / D, c = e - h * D;
-      S.qs[h][c >> 4][c & 15] = S.qf[h][c] * ks[c];
-    }
-    for (int h = warp; h < G; h += NW) {
-      float a = 0.f;
-      for (int c = lane; c < D; c += 32) a = fmaf(fabsf(S.qf[h][c]), ks[c], a);
-      a = nwarp_sum(a);
-      if (lane == 0) {
-        const float dl = 0.5f * a;
-        S.dmax[h] = fmaxf(S.dmax[h], dl);
-        sc.delta[(hrow0 + h) * sh.nbm + j] = dl;
+    // scaled queries of this block and Delta_b (base 2: sum |qs| / 2)
+#pragma unroll
+    for (int i = 0; i < NQI; ++i) {
+      const int e = tid + i * NT;
+      if (e - lane < QI) {  // warp-uniform
+        const bool act = e < QI;
+        const int h = act ? e / (D / 4) : 0, c = act ? 4 * (e % (D / 4)) : 0;
+        const float4 kq = *reinterpret_cast<const float4*>(ks + c);
+        const float4 qv = *reinterpret_cast<const float4*>(&S.qf[h][c]);
+        const float4 r = make_float4(qv.x * kq.x, qv.y * kq.y, qv.z * kq.z, qv.w * kq.w);
+        if (act) *reinterpret_cast<float4*>(&S.qs[k & 1][h][c / CH][c % CH]) = r;
+        float sa = act ? (fabsf(r.x) + fabsf(r.y)) + (fabsf(r.z) + fabsf(r.w)) : 0.f;
+#pragma unroll
+        for (int m = D / 8; m >= 1; m >>= 1) sa += __shfl_xor_sync(0xffffffffu, sa, m);
+        if (act && c == 0) {
+          S.dmax[h] = fmaxf(S.dmax[h], sa);  // one thread per head
+          if (trace) sc.delta[(hrow0 + h) * sh.nbm + j] = 0.5f * sa * LN2;
+        }
       }
     }
-    __syncthreads();
+    if (__syncthreads_or(!got)) {
+      ok = false;
+      break;
+    }
+    if (tid == 0 && k >= 1) {
+      fence_proxy_async_smem();
+      issue(k - 1 + NST);  // the previous block's stage is free
+    }
+    if (trace && k >= 1 && tid < G) {
+      float mm = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) mm = fmaxf(mm, S.ellp[(k - 1) & 1][w][tid]);
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) ss += exp2f(S.ellp[(k - 1) & 1][w][tid] - mm);
+      sc.ell8[(hrow0 + tid) * sh.nbm + j - 1] = (mm + log2f(ss)) * LN2;
+      if (tid == 0) sc.bflags[(size_t)unit * sh.nbm + j - 1] = 0;  // nothing promoted
+    }
 
-    // INT8 logits: warp w scores rows [w*8, w*8+8)
+    // ---- logits of the warp's 16 tokens: lane (tr, cc) scores rows tr + RPW*li ----
+    float x[NLI];
     {
-      float2 qs2[G][8];
+      float2 qr[G][CH / 2];  // register r: head r ^ pi
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        const float4* qp = reinterpret_cast<const float4*>(&S.qs[k & 1][r ^ pi][cc][0]);
+#pragma unroll
+        for (int i = 0; i < CH / 4; ++i) {
+          const float4 v = qp[i];
+          qr[r][2 * i] = make_float2(v.x, v.y);
+          qr[r][2 * i + 1] = make_float2(v.z, v.w);
+        }
+      }
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) {
+        const int row = warp * TPW + li * RPW + tr;
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(sp + (size_t)row * D + cc * CH);
+        uint32_t wd[CH / 4];
+        if constexpr (CH == 16) {
+          const uint4 v = *reinterpret_cast<const uint4*>(kw);
+          wd[0] = v.x; wd[1] = v.y; wd[2] = v.z; wd[3] = v.w;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(kw);
+          wd[0] = v.x; wd[1] = v.y;
+        }
+        float2 a2[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) a2[r] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int wi = 0; wi < CH / 4; ++wi) {
+          float2 x0, x1;
+          s8x4_f2(wd[wi], x0, x1);
+#pragma unroll
+          for (int r = 0; r < G; ++r) {
+            a2[r] = __ffma2_rn(qr[r][2 * wi], x0, a2[r]);
+            a2[r] = __ffma2_rn(qr[r][2 * wi + 1], x1, a2[r]);
+          }
+        }
+        float a[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) a[r] = a2[r].x + a2[r].y;
+        // reduce-scatter over the CPT lanes of the row: level m halves the heads held
+#pragma unroll
+        for (int m = CPT / 2, n = G; m >= 1; m >>= 1) {
+          if (n > 1) {
+#pragma unroll
+            for (int r = 0; r < G / 2; ++r)
+              if (r < n / 2) a[r] += __shfl_xor_sync(0xffffffffu, a[r + n / 2], m);
+            n >>= 1;
+          } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], m);
+          }
+        }
+        x[li] = a[0];  // head pi, row warp*TPW + li*RPW + tr
+      }
+    }
+
+    // ---- online softmax of head pi over the warp's tokens ----
+    float mb = x[0];
+#pragma unroll
+    for (int li = 1; li < NLI; ++li) mb = fmaxf(mb, x[li]);
+#pragma unroll
+    for (int m = CPT; m < 32; m <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, m));
+    const float mnew = fmaxf(mrun, mb);
+    const float alpha = ex2(mrun - mnew);  // 0 on the first block
+    float p[NLI], ps = 0.f;
+#pragma unroll
+    for (int li = 0; li < NLI; ++li) {
+      p[li] = ex2(x[li] - mnew);
+      ps += p[li];
+    }
+#pragma unroll
+    for (int m = CPT; m < 32; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
+    lrun = fmaf(lrun, alpha, ps);
+    erun = fmaf(erun, alpha, S.eta[stg] * ps);
+    mrun = mnew;
+    if (trace) {
+      float es = 0.f;
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) es += ex2(x[li] - mb);
+#pragma unroll
+      for (int m = CPT; m < 32; m <<= 1) es += __shfl_xor_sync(0xffffffffu, es, m);
+      if (owner) S.ellp[k & 1][warp][pi] = mb + log2f(es);
+    }
+    if (owner) S.alpha[warp][pi] = alpha;
+    const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+    // value scale folded into the weights; offset term accumulated here
+    if (dup * GPL < NG) {
+#pragma unroll
+      for (int i = 0; i < GPL; ++i) zl[i] *= alpha;
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) {
+        const int tok = li * RPW + tr;
+        const float* mrow = vm + ((size_t)(warp * TPW + tok) * NG + dup * GPL) * 2;
+#pragma unroll
+        for (int i = 0; i < GPL; ++i) {
+          const float2 sz = *reinterpret_cast<const float2*>(mrow + 2 * i);
+          S.ws[warp][tok][dup * GPL + i][pi] = p[li] * sz.x;
+          zl[i] = fmaf(p[li], sz.y, zl[i]);
+        }
+      }
+    }
+    __syncwarp();
+
+    // ---- P.V: lane (ts, cl) accumulates channels 8*cl .. 8*cl+7 of rows ts + TPI*i ----
+    if (rescale) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float4* qp = reinterpret_cast<const float4*>(&S.qs[h][cc][0]);
+        const float al = S.alpha[warp][h];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float4 x = qp[i];
-          qs2[h][2 * i] = make_float2(x.x, x.y);
-          qs2[h][2 * i + 1] = make_float2(x.z, x.w);
-        }
-      }
-#pragma unroll
-      for (int li = 0; li < NLW; ++li) {
-        const int r = warp * ROWS_PER_WARP + li * RPW + tr;
-        const uint4 ww = kc[r * CPT + cc];
-        float2 x[8];
-        s8x4_f2(ww.x, x[0], x[1]);
-        s8x4_f2(ww.y, x[2], x[3]);
-        s8x4_f2(ww.z, x[4], x[5]);
-        s8x4_f2(ww.w, x[6], x[7]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) a = __ffma2_rn(qs2[h][i], x[i], a);
-          float v = a.x + a.y;
-#pragma unroll
-          for (int m = CPT / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-          if (cc == 0) S.lg[h][r] = v;
+          acc[h][i].x *= al;
+          acc[h][i].y *= al;
         }
       }
     }
-    __syncthreads();
-    for (int h = warp; h < G; h += NW)
-      softmax_step(h, BLK, &sc.ell8[(hrow0 + h) * sh.nbm + j], S.eta[stg], false);
-    if (tid == 0) sc.bflags[(size_t)unit * sh.nbm + j] = 0;  // nothing promoted
-    __syncthreads();
-
-    // INT4 P.V with the per-group offset folded
-    pv_rescale();
 #pragma unroll
-    for (int p = 0; p < NPASS; ++p) {
-      const int tt = p * RPC + row;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(vc + (size_t)tt * (D / 2) + cl * 4);
-      const float2 meta = *reinterpret_cast<const float2*>(vm + ((size_t)tt * NG + (cl * 8) / VG) * 2);
+    for (int i = 0; i < NPI; ++i) {
+      const int tok = i * TPI + ts;
+      const uint32_t w =
+          *reinterpret_cast<const uint32_t*>(vc + (size_t)(warp * TPW + tok) * (D / 2) + cl * 4);
+      float wsv[G];
+      if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int h = 0; h < G; h += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(&S.ws[warp][tok][gq][h]);
+          wsv[h] = v.x; wsv[h + 1] = v.y; wsv[h + 2] = v.z; wsv[h + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h) wsv[h] = S.ws[warp][tok][gq][h];
+      }
       float2 cf[4];
-      u4x8_f2(w, cf);
+      u4x8_scaled(w, cf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pw = S.pp[h][tt];
-        const float ws = pw * meta.x;
-        zacc[h] = fmaf(pw, meta.y, zacc[h]);
+        const float2 ww = make_float2(wsv[h], wsv[h]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[h][i] = __ffma2_rn(make_float2(ws, ws), cf[i], acc[h][i]);
+        for (int q2 = 0; q2 < 4; ++q2) acc[h][q2] = __ffma2_rn(ww, cf[q2], acc[h][q2]);
       }
-    }
-    __syncthreads();  // the stage and S.pp are free again
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      issue(k + NST);
     }
   }
   if (!ok) {
-    for (int k2 = k + 1; k2 < k + NST && k2 < nblk; ++k2)
-      mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
-  }
-
-  // ---- partials ----
-  const size_t pbase = ((size_t)unit * sc.max_chunks + chunk) * G;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      S.red[row][cl * 8 + 2 * i] = acc[h][i].x + zacc[h];
-      S.red[row][cl * 8 + 2 * i + 1] = acc[h][i].y + zacc[h];
+    // let the copies still in flight land before the CTA exits
+    if (tid == 0) {
+      const int hi = min(nblk - 1, k == 0 ? NST - 1 : k + NST - 2);
+      for (int k2 = k; k2 <= hi; ++k2)
+        mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
     }
-    __syncthreads();
-    for (int c = tid; c < D; c += NT) {
-      float s = 0.f;
-      for (int r = 0; r < RPC; ++r) s += S.red[r][c];
-      sc.part_o[(pbase + h) * D + c] = s;
-    }
-    __syncthreads();
+    naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
+                             reinterpret_cast<float*>(dsm), &S.last);
+    return;
   }
-  if (tid < G) {
-    sc.part_s[(pbase + tid) * 3 + 0] = S.m[tid];
-    sc.part_s[(pbase + tid) * 3 + 1] = S.l[tid];
-    sc.part_s[(pbase + tid) * 3 + 2] = S.e[tid];
-    sc.part_x[(pbase + tid) * 3 + 0] = S.dmax[tid];
-    sc.part_x[(pbase + tid) * 3 + 1] = S.mres[tid];
-    sc.part_x[(pbase + tid) * 3 + 2] = S.lres[tid];
+  __syncthreads();  // every warp is past its last block: the stages are free
+  if (trace && nblk > 0 && tid < G) {
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mm = fmaxf(mm, S.ellp[(nblk - 1) & 1][w][tid]);
+    float ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ss += exp2f(S.ellp[(nblk - 1) & 1][w][tid] - mm);
+    sc.ell8[(hrow0 + tid) * sh.nbm + j0 + nblk - 1] = (mm + log2f(ss)) * LN2;
+    if (tid == 0) sc.bflags[(size_t)unit * sh.nbm + j0 + nblk - 1] = 0;
   }
-}
 
-__device__ double naive_e_key(double dT, double dA, double m8T) {
-  const double a = m8T * exp(dT);
-  const double m_ub = a > 0.0 ? a / (a + (1.0 - m8T) * exp(-dA)) : 0.0;
-  return fmin(tanh(0.5 * dT), m_ub * expm1(2.0 * dT));
-}
-
-// one CTA of D threads per (batch row, query head); thread c owns output channel c
-template <int D, int G>
-__global__ void naive_combine_kernel(DecodeShape sh, Scratch sc, int nchunks, int res_chunk,
-                                     float* __restrict__ out, float* __restrict__ e_key,
-                                     float* __restrict__ e_val, uint8_t* __restrict__ rung) {
-  constexpr int NW = D / 32;
-  __shared__ float wbuf[1024];
-  __shared__ float red[3][NW];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.x;
-  const int b = row / sh.Hq, h = row - b * sh.Hq;
-  const int g = h / G, hh = h - g * G;
-  const int unit = b * sh.Hkv + g;
-  const size_t base = (size_t)unit * sc.max_chunks * G + hh;
-  float ml = -INFINITY, dl = 0.f;
-  for (int c = tid; c < nchunks; c += D) {
-    ml = fmaxf(ml, sc.part_s[(base + (size_t)c * G) * 3]);
-    dl = fmaxf(dl, sc.part_x[(base + (size_t)c * G) * 3]);
+  // ---- merge the four warps' states ----
+  float* ow = reinterpret_cast<float*>(dsm);  // [NW][G][D] unscaled P.V of each warp
+  float* zw = ow + NW * G * D;                // [NW][G][NG] offset terms
+  float* mw = zw + NW * G * NG;               // [NW][G][3] m, l, e
+#pragma unroll
+  for (int m = LPT; m < 32; m <<= 1)
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[h][i].x += __shfl_xor_sync(0xffffffffu, acc[h][i].x, m);
+        acc[h][i].y += __shfl_xor_sync(0xffffffffu, acc[h][i].y, m);
+      }
+  if (ts == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float2*>(&ow[(warp * G + h) * D + cl * 8 + 2 * i]) =
+            make_float2(acc[h][i].x * nib_unscale(2 * i), acc[h][i].y * nib_unscale(2 * i + 1));
   }
-  ml = nwarp_max(ml);
-  dl = nwarp_max(dl);
-  if (lane == 0) {
-    red[0][warp] = ml;
-    red[1][warp] = dl;
+#pragma unroll
+  for (int m = CPT; m < 32; m <<= 1)
+#pragma unroll
+    for (int i = 0; i < GPL; ++i) zl[i] += __shfl_xor_sync(0xffffffffu, zl[i], m);
+  if (tr == 0 && dup * GPL < NG) {
+#pragma unroll
+    for (int i = 0; i < GPL; ++i) zw[(warp * G + pi) * NG + dup * GPL + i] = zl[i];
+  }
+  if (owner) {
+    mw[(warp * G + pi) * 3 + 0] = mrun;
+    mw[(warp * G + pi) * 3 + 1] = lrun;
+    mw[(warp * G + pi) * 3 + 2] = erun;
   }
   __syncthreads();
-  float M = -INFINITY, dA = 0.f;
+  for (int e = tid; e < G * D; e += NT) {
+    const int h = e / D, c = e - h * D;
+    float M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    M = fmaxf(M, red[0][w]);
-    dA = fmaxf(dA, red[1][w]);
-  }
-  __syncthreads();
-  float ll = 0.f, el = 0.f;
-  for (int c = tid; c < nchunks; c += D) {
-    const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
-    const float w = ps[0] == -INFINITY ? 0.f : expf(ps[0] - M);
-    if (c < 1024) wbuf[c] = w;
-    ll += ps[1] * w;
-    el += ps[2] * w;
-  }
-  ll = nwarp_sum(ll);
-  el = nwarp_sum(el);
-  if (lane == 0) {
-    red[0][warp] = ll;
-    red[1][warp] = el;
-  }
-  __syncthreads();
-  float L = 0.f, E = 0.f;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[(w * G + h) * 3]);
+    float o = 0.f;
+    if (M != -INFINITY) {
 #pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    L += red[0][w];
-    E += red[1][w];
-  }
-  // o: batches of 16 independent loads so the chain of chunk partials does not
-  // serialise on memory latency
-  float o = 0.f;
-  for (int c0 = 0; c0 < nchunks; c0 += 16) {
-    float v[16], wv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = c0 + i;
-      v[i] = 0.f;
-      wv[i] = 0.f;
-      if (c < nchunks) {
-        const size_t pi = base + (size_t)c * G;
-        v[i] = sc.part_o[pi * D + tid];
-        if (c < 1024) {
-          wv[i] = wbuf[c];
-        } else {
-          const float mc = sc.part_s[pi * 3];
-          wv[i] = mc == -INFINITY ? 0.f : expf(mc - M);
-        }
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(mw[(w * G + h) * 3] - M);
+        o = fmaf(f, ow[(w * G + h) * D + c] + zw[(w * G + h) * NG + c / VG], o);
       }
     }
+    sc.part_o[(pbase + h) * D + c] = o;
+  }
+  if (tid < G) {
+    float M = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) o = fmaf(v[i], wv[i], o);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mw[(w * G + tid) * 3]);
+    float L = 0.f, E = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(mw[(w * G + tid) * 3] - M);
+        L = fmaf(f, mw[(w * G + tid) * 3 + 1], L);
+        E = fmaf(f, mw[(w * G + tid) * 3 + 2], E);
+      }
+    }
+    sc.part_s[(pbase + tid) * 3 + 0] = M == -INFINITY ? -INFINITY : M * LN2;
+    sc.part_s[(pbase + tid) * 3 + 1] = L;
+    sc.part_s[(pbase + tid) * 3 + 2] = E;
+    sc.part_x[(pbase + tid) * 3 + 0] = 0.5f * S.dmax[tid] * LN2;
+    sc.part_x[(pbase + tid) * 3 + 1] = -INFINITY;
+    sc.part_x[(pbase + tid) * 3 + 2] = 0.f;
   }
-  out[(size_t)row * D + tid] = o / L;
-  if (tid == 0) {
-    // the residual CTA holds the residual's own statistics
-    const float* px = sc.part_x + (base + (size_t)res_chunk * G) * 3;
-    const double mres = px[1] == -INFINITY ? 0.0 : (double)px[2] * exp((double)px[1] - M) / L;
-    const double m8T = 1.0 - mres;
-    const float ek = sh.nb > 0 ? (float)naive_e_key((double)dA, (double)dA, m8T) : 0.f;
-    e_key[row] = ek;
-    e_val[row] = E / L;
-    rung[row] = 0;
-    sc.ekey[row] = ek;
-    sc.hflags[row] = 0;
-    sc.kstar[row] = 0;
-    sc.dense[row] = 0;
-  }
+  naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
+                           reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::MAIN, &S.last);
 }
 
 // chunking of the streaming pass: about four resident CTAs per SM over all units
@@ -495,19 +752,19 @@ void naive_chunking(const DecodeShape& sh, int max_chunks, int* cb, int* nch) {
 template <int D, int G>
 cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                     const __half* q, const Scratch& sc, float* out, float* e_key, float* e_val,
-                    uint8_t* rung, int part, cudaStream_t s) {
+                    uint8_t* rung, int trace, cudaStream_t s) {
   int cb, nch;
   naive_chunking(sh, sc.max_chunks, &cb, &nch);
-  if (part == 0) {
-    const int smem = NST * NaiveLayout<D>::STAGE;
-    cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G>, (int)smem);
-    if (e != cudaSuccess) return e;
-    naive_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc,
-                                                                      cb, nch);
-    return cudaGetLastError();
-  }
-  naive_combine_kernel<D, G><<<sh.B * sh.Hq, D, 0, s>>>(sh, sc, nch + 1, nch, out, e_key, e_val,
-                                                          rung);
+  const int smem = NST * NaiveLayout<D>::STAGE;
+  // the merge keeps (nch + 1) * G weights, G inverse sums and NT float4 partial
+  // sums in the stage area, after what the CTAs still hold there
+  const size_t merge_floats =
+      (size_t)NaiveMergeAt<D, G>::AT + (size_t)(nch + 1) * G + G + 4 + (size_t)NT * 4;
+  if (merge_floats * 4 > (size_t)smem) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G>, (int)smem);
+  if (e != cudaSuccess) return e;
+  naive_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(
+      t, st, unit0, sh, q, sc, cb, nch, trace, out, e_key, e_val, rung);
   return cudaGetLastError();
 }
 
@@ -515,9 +772,9 @@ cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeSh
 
 cudaError_t launch_naive(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                          const __half* q, const Scratch& sc, float* out, float* e_key,
-                         float* e_val, uint8_t* rung, int part, cudaStream_t s) {
+                         float* e_val, uint8_t* rung, int trace, cudaStream_t s) {
 #define CQA_NAIVE_CASE(DD, GG) \
-  return naive_t<DD, GG>(t, st, unit0, sh, q, sc, out, e_key, e_val, rung, part, s)
+  return naive_t<DD, GG>(t, st, unit0, sh, q, sc, out, e_key, e_val, rung, trace, s)
   if (sh.d == 128) {
     switch (sh.G) {
       case 1: CQA_NAIVE_CASE(128, 1);

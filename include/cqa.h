@@ -118,8 +118,10 @@ int cqa_cache_length(const cqa_cache* cache, int layer, int32_t* out_len);
  * fp32 scale per (block, channel) (s = amax/127, code = round-half-even(k/s)),
  * values -> asymmetric INT4 per (token, 32 channels) (z = min,
  * s = (max-min)/15), eta_b = max |v - (s*code + z)| over the block; the newest
- * length % 64 tokens stay exact in FP16 (the residual block).  All appended
- * tokens are also written to Tier 2.  The encoding of a block depends only on
+ * length % 64 tokens stay exact in FP16 (the residual block, device memory).
+ * A block's FP16 originals are written to Tier 2 when it seals (the residual
+ * block is never promoted, so its tokens need no host copy before that).
+ * The encoding of a block depends only on
  * its tokens, so appending in any chunking gives the same cache.
  * CQA_ERR_CAPACITY if length + n_new > max_ctx.  n_new = 0 is a no-op. */
 int cqa_quantize_append(cqa_cache* cache, int layer, const void* k_fp16, const void* v_fp16,
@@ -155,7 +157,8 @@ int cqa_dense_reference(cqa_cache* cache, int layer, const void* q_fp16, float* 
  *   CQA_EXPORT_ETA      fp32  [batch][n_kv_heads][nb]
  *   CQA_EXPORT_VRANGE   fp32  [batch][n_kv_heads][2][d]  (vmin, vmax over all tokens)
  *   CQA_EXPORT_RESIDUAL fp16  [batch][n_kv_heads][2][length % 64][d]  (keys, values)
- *   CQA_EXPORT_TIER2    fp16  [batch][n_kv_heads][2][length][d]  (keys, values)
+ *   CQA_EXPORT_TIER2    fp16  [batch][n_kv_heads][2][length][d]  (keys, values: the
+ *                       sealed tokens from Tier 2, the residual block's from device)
  * `bytes` must equal the array's size (CQA_ERR_INVALID_ARG otherwise);
  * cqa_debug_export(cache, layer, what, NULL, 0) returns that size instead
  * (as a non-negative value, or a negative error). */
@@ -205,8 +208,8 @@ int cqa_set_key_prefetch(cqa_cache* cache, int mode, float min_fraction);
  * them and reports, per phase, the summed event time in milliseconds and the
  * number of kernel launches.  Phases: */
 enum {
-  CQA_PHASE_APPEND_SEAL = 0,   /* sealing complete blocks into Tier 1 */
-  CQA_PHASE_APPEND_TAIL = 1,   /* Tier-2 copy, residual block, value ranges */
+  CQA_PHASE_APPEND_SEAL = 0,   /* sealing complete blocks into Tier 1 and Tier 2 */
+  CQA_PHASE_APPEND_TAIL = 1,   /* residual block, value ranges */
   CQA_PHASE_SCORE = 2,         /* INT8 scoring pass */
   CQA_PHASE_SELECT = 3,        /* coverage selection, E_key, rungs 1-2 */
   CQA_PHASE_PROMOTE = 4,       /* FP16 keys of promoted blocks from Tier 2: exact logits */
@@ -217,8 +220,9 @@ enum {
   CQA_PHASE_DENSE_ATTEND = 9,  /* exact attention from Tier 2 (E_val post-check, reference) */
   CQA_PHASE_DENSE_COMBINE = 10,
   CQA_PHASE_PREFETCH = 11,     /* copy-engine copy of a layer's Tier-2 keys (not a kernel) */
-  CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1 */
-  CQA_PHASE_NAIVE_COMBINE = 13,
+  CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1, whose
+                                  last CTA per (batch row, kv head) also combines */
+  CQA_PHASE_NAIVE_COMBINE = 13, /* reserved: no separate launch (the pass combines) */
   CQA_PHASE_COUNT = 14
 };
 /* Start (or restart) profiling; max_launches bounds the recorded launches
