@@ -12,11 +12,22 @@
 //   ell8_b  = log sum_{t in b} exp(logit_t)
 //   Delta_b = sigma/2 * sum_c |q_c| * s_c               (|k - s*code| <= s/2)
 //
-// The pass streams 136 bytes per token and kv head (128 B of codes, 8 B of
-// scales amortised) from HBM and writes 16 B of logits; it is bound by HBM
-// bandwidth and, close behind, by fp32 issue rate, so codes are widened with
-// a byte-permute into the mantissa of 2^23 and the dot products use packed
-// float2 FMAs.
+// The pass reads 136 bytes per token and kv head (128 B of codes, 8 B of
+// scales amortised) and writes 16 B of logits.  Its cost is instruction issue
+// as much as HBM, so it is laid out like the certification-off pass:
+//   * one CTA streams consecutive blocks of one (batch row, kv head) through
+//     a ring of NST stages filled by bulk copies (codes + scales of a block);
+//   * one CTA barrier per block publishes the block's scaled queries
+//     (q * sigma * s_c, double-buffered by block parity) and releases the
+//     previous block's stage;
+//   * each warp scores 16 tokens of every block: sixteen lanes per token,
+//     8 channels each, packed float2 FMAs, the G partial dots reduced with a
+//     reduce-scatter whose register order is permuted per lane;
+//   * each warp reduces its tokens' log-sum-exp per head; the four slices
+//     merge into ell8_b after the next barrier;
+//   * logits leave through shared memory as 16-byte stores.
+// The residual block is scored exactly from its FP16 keys by one more CTA per
+// (batch row, kv head).
 #include "bulk_pipe.cuh"
 #include "cqa_internal.cuh"
 
@@ -24,7 +35,32 @@ namespace cqa {
 
 namespace {
 
-constexpr int WARPS = 4;
+constexpr int NT = 128;  // threads per CTA: four warps
+constexpr int NW = NT / 32;
+constexpr int NST = 4;         // stages per CTA
+constexpr int TPW = BLK / NW;  // tokens of each block scored by one warp
+constexpr int CH = 8;          // channels per lane
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int D>
+struct ScoreLayout {
+  static constexpr int KB = BLK * D;  // INT8 key codes
+  static constexpr int SB = 4 * D;    // key scales
+  static constexpr int STAGE = KB + SB;
+};
+
+__device__ __forceinline__ float swarp_max(float x) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
+  return x;
+}
+
+__device__ __forceinline__ float swarp_sum(float x) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
+}
 
 // Four signed int8 codes -> two float2, exactly: bias to unsigned, drop each
 // byte into the low mantissa bits of 2^23, subtract 2^23 + 128.
@@ -39,272 +75,284 @@ __device__ __forceinline__ void s8x4_to_f2(uint32_t w, float2& a, float2& b) {
                  off);
 }
 
-// v[i] holds N partial sums on each of the N lanes of an aligned lane group;
-// afterwards lane l of the group holds the full sum of value index (l % N).
-template <int N>
-__device__ __forceinline__ float reduce_scatter(float (&v)[N], int lane) {
-#pragma unroll
-  for (int m = N / 2; m >= 1; m >>= 1) {
-    const bool hi = (lane & m) != 0;
-#pragma unroll
-    for (int i = 0; i < m; ++i) {
-      const float send = hi ? v[i] : v[i + m];
-      const float keep = hi ? v[i + m] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-    }
-  }
-  return v[0];
+// 2^x by the hardware approximation (relative error about 2^-22)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
-  return x;
-}
-
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
-  return x;
-}
-
-// Warp-level pipeline: each warp streams its (unit, block) items through
-// NSTAGE shared-memory stages filled by bulk copies (codes + scales of one
-// block per stage), so several blocks are in flight per warp without holding
-// them in registers.  Item k of warp gw is the sealed item gw + k * nw; warps
-// gw < units first compute the residual block of unit gw while their first
-// copies land.
-constexpr int NSTAGE = 2;
-
-template <int D>
-__host__ __device__ constexpr int stage_bytes() { return BLK * D + 4 * D; }
 
 template <int D, int G>
-__global__ void __launch_bounds__(WARPS * 32, 3)
+struct ScoreSmem {
+  float qf[G][D];                   // q * sigma
+  float qs[2][G][D / CH][CH + 4];   // qf * key scale of the block, by block parity; rows padded
+                                    // by 4 floats so eight lanes' 16-byte reads hit distinct banks
+  float lgs[NW][G][TPW];            // each warp's logits of the current block
+  float ellp[2][NW][G][2];          // each warp's (max, sum of 2^((x - max) log2 e)) per head
+  uint64_t bar[NST];
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(NT, 5)
     score_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
-                 Scratch sc, int n_sealed, int n_res) {
-  constexpr int CPT = D / 16;    // lanes per token row (16 channels each)
-  constexpr int RPW = 32 / CPT;  // rows covered by one warp-wide 16-byte load
-  constexpr int NL = BLK / RPW;  // loads per lane per block
-  constexpr int R = CPT / G;     // rows per reduce-scatter round
-  constexpr int SB = stage_bytes<D>();
-  static_assert(R >= 1 && NL % R == 0, "unsupported head_dim / group size");
+                 Scratch sc, int chunk_blocks, int nres_chunk) {
+  using LY = ScoreLayout<D>;
+  constexpr int CPT = D / CH;     // lanes per token row
+  constexpr int RPW = 32 / CPT;   // rows per warp instruction
+  constexpr int NLI = TPW / RPW;  // logit iterations per block
+  constexpr int NDUP = CPT > G ? CPT / G : 1;
+  constexpr int QI = G * D / 4;   // float4 items of the scaled queries
+  constexpr int NQI = (QI + NT - 1) / NT;
+  static_assert(NLI >= 1 && RPW * NLI == TPW, "layout");
 
   extern __shared__ __align__(128) unsigned char dsm[];
-  __shared__ __align__(16) float lg[WARPS][G][BLK];
-  __shared__ __align__(8) uint64_t bars[WARPS][NSTAGE];
+  __shared__ __align__(16) ScoreSmem<D, G> S;
 
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int cc = lane % CPT, tr = lane / CPT;
-  const int nw = gridDim.x * WARPS;
-  const int gw = blockIdx.x * WARPS + wib;
-  unsigned char* wstage = dsm + (size_t)wib * NSTAGE * SB;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int unit = blockIdx.y;
+  const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
+  const size_t u = (size_t)unit0 + unit;
+  const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
+  const int chunk = blockIdx.x;
 
-  if (lane == 0) {
-    for (int s2 = 0; s2 < NSTAGE; ++s2) mbar_init(&bars[wib][s2], 1);
+  for (int e = tid; e < G * D; e += NT) {
+    const int h = e / D, c = e - h * D;
+    S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * sh.sigma;
+  }
+
+  // ---- the residual block: exact logits from the FP16 keys in device memory ----
+  if (chunk == nres_chunk) {
+    __syncthreads();
+    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK]
+    const int r = sh.r;
+    const __half* kr = t.kres + u * st.res;
+    constexpr int CPL = D / 32;
+    for (int tt = warp; tt < r; tt += NW) {
+      float kf[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; i += 2) {
+        const float2 f = __half22float2(
+            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
+        kf[i] = f.x;
+        kf[i + 1] = f.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
+        v = swarp_sum(v);
+        if (lane == 0) lg[h * BLK + tt] = v;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += NW) {
+      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
+      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
+      float* lo = sc.logits + (hrow0 + h) * sc.ls + (size_t)sh.nb * BLK;
+      if (lane < r) lo[lane] = x0;
+      if (lane + 32 < r) lo[lane + 32] = x1;
+      float lse = -INFINITY;
+      if (r > 0) {
+        const float m = swarp_max(fmaxf(x0, x1));
+        const float ssum = swarp_sum((lane < r ? expf(x0 - m) : 0.f) +
+                                     (lane + 32 < r ? expf(x1 - m) : 0.f));
+        lse = m + logf(ssum);
+      }
+      if (lane == 0) sc.ell_res[hrow0 + h] = lse;
+    }
+    return;
+  }
+
+  const int j0 = chunk * chunk_blocks;
+  const int nblk = max(0, min(sh.nb, j0 + chunk_blocks) - j0);
+  if (tid == 0) {
+    for (int s2 = 0; s2 < NST; ++s2) mbar_init(&S.bar[s2], 1);
     mbar_init_fence();
   }
-  __syncwarp();
+  __syncthreads();
 
-  auto issue = [&](int k) {  // lane 0: start the copies of this warp's k-th item
-    const int it = gw + k * nw;
-    if (it >= n_sealed) return;
-    const int unit = it / sh.nb, j = it - unit * sh.nb;
-    const size_t u = (size_t)unit0 + unit;
-    uint64_t* bar = &bars[wib][k % NSTAGE];
-    unsigned char* dst = wstage + (size_t)(k % NSTAGE) * SB;
-    mbar_arrive_expect_tx(bar, SB);
-    bulk_g2s(dst, t.kcodes + u * st.kcodes + (size_t)j * BLK * D, BLK * D, bar);
-    bulk_g2s(dst + BLK * D, t.kscale + u * st.kscale + (size_t)j * D, 4 * D, bar);
+  auto issue = [&](int k) {  // thread 0: copies of the chunk's k-th block
+    if (k >= nblk) return;
+    const int j = j0 + k;
+    unsigned char* dst = dsm + (size_t)(k % NST) * LY::STAGE;
+    uint64_t* bar = &S.bar[k % NST];
+    mbar_arrive_expect_tx(bar, LY::STAGE);
+    bulk_g2s(dst, t.kcodes + u * st.kcodes + (size_t)j * LY::KB, LY::KB, bar);
+    bulk_g2s(dst + LY::KB, t.kscale + u * st.kscale + (size_t)j * D, LY::SB, bar);
   };
-  if (lane == 0)
-    for (int k = 0; k < NSTAGE; ++k) issue(k);
+  if (tid == 0)
+    for (int k = 0; k < NST; ++k) issue(k);
 
-  if (gw < n_res) {
-    const int it = n_sealed + gw;
-    // residual block: exact logits from the FP16 keys kept in device memory;
-      // LPR lanes per token row, 8 channels each
-      constexpr int LPR = D / 8;
-      constexpr int RW = 32 / LPR;  // rows per warp pass
-      const int unit = it - n_sealed;
-      const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
-      const size_t u = (size_t)unit0 + unit;
-      const int cl = lane % LPR, rl = lane / LPR;
-      const __half* kr = t.kres + u * st.res;
-      float2 qf[G][4];
+  // ell8 of block j from the four warps' slices
+  auto finish_ell = [&](int pbuf, int j) {
+    if (tid < G) {
+      float mm = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(
-            q + ((size_t)b * sh.Hq + (size_t)g * G + h) * D + cl * 8));
-        const __half2* qh = reinterpret_cast<const __half2*>(&qv);
+      for (int w = 0; w < NW; ++w) mm = fmaxf(mm, S.ellp[pbuf][w][tid][0]);
+      float ss = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) qf[h][k] = __half22float2(qh[k]);
-      }
-      for (int r0 = 0; r0 < sh.r; r0 += RW) {
-        const int tok = r0 + rl;
-        float2 kf[4];
-        if (tok < sh.r) {
-          const uint4 kv = *reinterpret_cast<const uint4*>(kr + (size_t)tok * D + cl * 8);
-          const __half2* kh = reinterpret_cast<const __half2*>(&kv);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) kf[k] = __half22float2(kh[k]);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) kf[k] = make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) a = __ffma2_rn(qf[h][k], kf[k], a);
-          float v = a.x + a.y;
-#pragma unroll
-          for (int m = LPR / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-          if (cl == 0 && tok < sh.r) lg[wib][h][tok] = v * sh.sigma;
-        }
-      }
-      __syncwarp();
-#pragma unroll 1
-      for (int h = 0; h < G; ++h) {
-        const float x0 = lane < sh.r ? lg[wib][h][lane] : -INFINITY;
-        const float x1 = lane + 32 < sh.r ? lg[wib][h][lane + 32] : -INFINITY;
-        float* lo = sc.logits + ((size_t)b * sh.Hq + (size_t)g * G + h) * sc.ls + (size_t)sh.nb * BLK;
-        if (lane < sh.r) lo[lane] = x0;
-        if (lane + 32 < sh.r) lo[lane + 32] = x1;
-        float lse = -INFINITY;
-        if (sh.r > 0) {
-          const float m = warp_max(fmaxf(x0, x1));
-          const float ssum = warp_sum((x0 > -INFINITY ? expf(x0 - m) : 0.f) +
-                                      (x1 > -INFINITY ? expf(x1 - m) : 0.f));
-          lse = m + logf(ssum);
-        }
-        if (lane == 0) sc.ell_res[(size_t)b * sh.Hq + (size_t)g * G + h] = lse;
-      }
-      __syncwarp();
-  }
+      for (int w = 0; w < NW; ++w)
+        ss += S.ellp[pbuf][w][tid][1] * ex2((S.ellp[pbuf][w][tid][0] - mm) * LOG2E);
+      sc.ell8[(hrow0 + tid) * sh.nbm + j] = mm + log2f(ss) * LN2;
+    }
+  };
 
-  int k = 0;
+  const int cc = lane % CPT, tr = lane / CPT;  // channel slice, row
+  int pi = 0;                                  // head permutation of the reduce-scatter
+#pragma unroll
+  for (int m = CPT / 2, n = G; m >= 1; m >>= 1, n >>= 1)
+    if (n > 1 && (cc & m)) pi |= n / 2;
+  const bool owner = tr == 0 && (cc & (NDUP - 1)) == 0;  // one lane per head of the warp
+
   bool ok = true;
-  for (; gw + k * nw < n_sealed; ++k) {
-    const int it = gw + k * nw;
-    const int stg = k % NSTAGE;
-    ok = mbar_wait(&bars[wib][stg], (uint32_t)((k / NSTAGE) & 1), sc.err);
-    if (!ok) break;
-    const uint4* stage_codes = reinterpret_cast<const uint4*>(wstage + (size_t)stg * SB);
-    const float* stage_scales = reinterpret_cast<const float*>(wstage + (size_t)stg * SB + BLK * D);
-    {
-      const int unit = it / sh.nb, j = it - unit * sh.nb;
-      const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
-      float s[16];
-      {
-        const float4* sp = reinterpret_cast<const float4*>(stage_scales + cc * 16);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 x = sp[i];
-          s[4 * i] = x.x;
-          s[4 * i + 1] = x.y;
-          s[4 * i + 2] = x.z;
-          s[4 * i + 3] = x.w;
-        }
-      }
-      float2 qs[G][8];
-      float dp[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint4* qp = reinterpret_cast<const uint4*>(
-            q + ((size_t)b * sh.Hq + (size_t)g * G + h) * D + cc * 16);
-        uint4 qa = __ldg(qp), qb = __ldg(qp + 1);
-        const __half2* qh0 = reinterpret_cast<const __half2*>(&qa);
-        const __half2* qh1 = reinterpret_cast<const __half2*>(&qb);
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 qf = __half22float2(k < 4 ? qh0[k] : qh1[k - 4]);
-          acc = fmaf(fabsf(qf.x), s[2 * k], acc);
-          acc = fmaf(fabsf(qf.y), s[2 * k + 1], acc);
-          qs[h][k] = make_float2(qf.x * s[2 * k] * sh.sigma, qf.y * s[2 * k + 1] * sh.sigma);
-        }
-        dp[h] = acc;
-      }
+  int k = 0;
+  for (; k < nblk; ++k) {
+    const int j = j0 + k;
+    const int stg = k % NST;
+    const bool got = mbar_wait(&S.bar[stg], (uint32_t)((k / NST) & 1), sc.err);
+    const unsigned char* sp = dsm + (size_t)stg * LY::STAGE;
+    const float* ks = reinterpret_cast<const float*>(sp + LY::KB);
 
+    // scaled queries of this block and Delta_b = sum |qs| / 2
 #pragma unroll
-      for (int i0 = 0; i0 < NL; i0 += R) {
-        float v[CPT];
+    for (int i = 0; i < NQI; ++i) {
+      const int e = tid + i * NT;
+      if (e - lane < QI) {  // warp-uniform
+        const bool act = e < QI;
+        const int h = act ? e / (D / 4) : 0, c = act ? 4 * (e % (D / 4)) : 0;
+        const float4 kq = *reinterpret_cast<const float4*>(ks + c);
+        const float4 qv = *reinterpret_cast<const float4*>(&S.qf[h][c]);
+        const float4 r = make_float4(qv.x * kq.x, qv.y * kq.y, qv.z * kq.z, qv.w * kq.w);
+        if (act) *reinterpret_cast<float4*>(&S.qs[k & 1][h][c / CH][c % CH]) = r;
+        float sa = act ? (fabsf(r.x) + fabsf(r.y)) + (fabsf(r.z) + fabsf(r.w)) : 0.f;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint4 ww = stage_codes[(i0 + r) * 32 + lane];
-          float2 x[8];
-          s8x4_to_f2(ww.x, x[0], x[1]);
-          s8x4_to_f2(ww.y, x[2], x[3]);
-          s8x4_to_f2(ww.z, x[4], x[5]);
-          s8x4_to_f2(ww.w, x[6], x[7]);
+        for (int m = D / 8; m >= 1; m >>= 1) sa += __shfl_xor_sync(0xffffffffu, sa, m);
+        if (act && c == 0) sc.delta[(hrow0 + h) * sh.nbm + j] = 0.5f * sa;
+      }
+    }
+    if (__syncthreads_or(!got)) {
+      ok = false;
+      break;
+    }
+    if (tid == 0 && k >= 1) {
+      fence_proxy_async_smem();
+      issue(k - 1 + NST);  // the previous block's stage is free
+    }
+    if (k >= 1) finish_ell((k - 1) & 1, j - 1);
+
+    // ---- logits of the warp's 16 tokens: lane (tr, cc) scores rows tr + RPW*li ----
+    float x[NLI];
+    {
+      float2 qr[G][CH / 2];  // register r: head r ^ pi
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float2 a = make_float2(0.f, 0.f);
+      for (int r = 0; r < G; ++r) {
+        const float4* qp = reinterpret_cast<const float4*>(&S.qs[k & 1][r ^ pi][cc][0]);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) a = __ffma2_rn(qs[h][k], x[k], a);
-            v[r * G + h] = a.x + a.y;
+        for (int i = 0; i < CH / 4; ++i) {
+          const float4 v = qp[i];
+          qr[r][2 * i] = make_float2(v.x, v.y);
+          qr[r][2 * i + 1] = make_float2(v.z, v.w);
+        }
+      }
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) {
+        const int row = warp * TPW + li * RPW + tr;
+        const uint2 wd = *reinterpret_cast<const uint2*>(sp + (size_t)row * D + cc * CH);
+        float2 k0, k1, k2, k3;
+        s8x4_to_f2(wd.x, k0, k1);
+        s8x4_to_f2(wd.y, k2, k3);
+        float a[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+          float2 a2 = __fmul2_rn(qr[r][0], k0);
+          a2 = __ffma2_rn(qr[r][1], k1, a2);
+          a2 = __ffma2_rn(qr[r][2], k2, a2);
+          a2 = __ffma2_rn(qr[r][3], k3, a2);
+          a[r] = a2.x + a2.y;
+        }
+        // reduce-scatter over the CPT lanes of the row: level m halves the heads held
+#pragma unroll
+        for (int m = CPT / 2, n = G; m >= 1; m >>= 1) {
+          if (n > 1) {
+#pragma unroll
+            for (int r = 0; r < G / 2; ++r)
+              if (r < n / 2) a[r] += __shfl_xor_sync(0xffffffffu, a[r + n / 2], m);
+            n >>= 1;
+          } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], m);
           }
         }
-        const float full = reduce_scatter<CPT>(v, lane);
-        const int rr = cc / G, hh = cc - rr * G;
-        lg[wib][hh][RPW * (i0 + rr) + tr] = full;
+        x[li] = a[0];  // head pi, row warp*TPW + li*RPW + tr
       }
-      // Delta: reduce the per-lane channel partials over the row's lanes
+    }
+
+    // ---- the warp's slice of ell8 and its logits ----
+    float mb = x[0];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+    for (int li = 1; li < NLI; ++li) mb = fmaxf(mb, x[li]);
 #pragma unroll
-        for (int m = CPT / 2; m >= 1; m >>= 1) dp[h] += __shfl_xor_sync(0xffffffffu, dp[h], m);
-      }
-      __syncwarp();
+    for (int m = CPT; m < 32; m <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, m));
+    const float mb2 = mb * LOG2E;
+    float es = 0.f;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float x0 = lg[wib][h][lane], x1 = lg[wib][h][lane + 32];
-        const float m = warp_max(fmaxf(x0, x1));
-        const float ssum = warp_sum(expf(x0 - m) + expf(x1 - m));
-        if (lane == 0) {
-          const size_t row = ((size_t)b * sh.Hq + (size_t)g * G + h) * sh.nbm + j;
-          sc.ell8[row] = m + logf(ssum);
-          sc.delta[row] = 0.5f * sh.sigma * dp[h];
-        }
-      }
-      float* lo = sc.logits + ((size_t)b * sh.Hq + (size_t)g * G) * sc.ls + (size_t)j * BLK;
-      for (int e = lane; e < G * (BLK / 4); e += 32) {
-        const int h = e / (BLK / 4), k = e - h * (BLK / 4);
-        *reinterpret_cast<float4*>(lo + h * sc.ls + 4 * k) =
-            *reinterpret_cast<const float4*>(&lg[wib][h][4 * k]);
-      }
-      __syncwarp();
+    for (int li = 0; li < NLI; ++li) es += ex2(fmaf(x[li], LOG2E, -mb2));
+#pragma unroll
+    for (int m = CPT; m < 32; m <<= 1) es += __shfl_xor_sync(0xffffffffu, es, m);
+    if (owner) {
+      S.ellp[k & 1][warp][pi][0] = mb;
+      S.ellp[k & 1][warp][pi][1] = es;
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) S.lgs[warp][pi][li * RPW + tr] = x[li];
+    }
+    if (tr > 0 && (cc & (NDUP - 1)) == 0) {
+#pragma unroll
+      for (int li = 0; li < NLI; ++li) S.lgs[warp][pi][li * RPW + tr] = x[li];
     }
     __syncwarp();
-    if (lane == 0) {
-      fence_proxy_async_smem();
-      issue(k + NSTAGE);
+    if (lane < G * TPW / 4) {
+      const int h = lane / (TPW / 4), t4 = lane % (TPW / 4);
+      const float4 v = *reinterpret_cast<const float4*>(&S.lgs[warp][h][4 * t4]);
+      *reinterpret_cast<float4*>(sc.logits + (hrow0 + h) * sc.ls + (size_t)j * BLK +
+                                 warp * TPW + 4 * t4) = v;
     }
+    __syncwarp();
   }
-  if (!ok) {
-    // a copy did not land in time: wait (bounded) for the ones still in flight
-    for (int k2 = k + 1; k2 < k + NSTAGE && gw + k2 * nw < n_sealed; ++k2)
-      mbar_wait(&bars[wib][k2 % NSTAGE], (uint32_t)((k2 / NSTAGE) & 1), nullptr);
+  if (__syncthreads_or(!ok)) {
+    // let the copies still in flight land before the CTA exits
+    if (tid == 0) {
+      const int hi = min(nblk - 1, k == 0 ? NST - 1 : k + NST - 2);
+      for (int k2 = k; k2 <= hi; ++k2)
+        mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
+    }
+    return;
   }
+  if (nblk > 0) finish_ell((nblk - 1) & 1, j0 + nblk - 1);
+}
+
+// chunking: about five resident CTAs per SM over all units, one more per unit
+// for the residual block
+void score_chunking(const DecodeShape& sh, int* cb, int* nch) {
+  const int units = sh.B * sh.Hkv;
+  int per_unit = (148 * 5 + units - 1) / units;
+  if (per_unit < 1) per_unit = 1;
+  int c = sh.nb > 0 ? (sh.nb + per_unit - 1) / per_unit : 1;
+  if (c < 1) c = 1;
+  const int n = sh.nb > 0 ? (sh.nb + c - 1) / c : 0;
+  *cb = c;
+  *nch = n;
 }
 
 template <int D, int G>
 cudaError_t launch_score_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                            const __half* q, const Scratch& sc, cudaStream_t s) {
-  const int units = sh.B * sh.Hkv;
-  const int n_sealed = units * sh.nb;
-  // enough warps for every residual item, at most three resident CTAs per SM
-  int grid = (n_sealed + 2 * WARPS - 1) / (2 * WARPS);
-  const int cap = 148 * 3;
-  if (grid > cap) grid = cap;
-  const int need_res = (units + WARPS - 1) / WARPS;
-  if (grid < need_res) grid = need_res;
-  if (grid < 1) grid = 1;
-  const int smem = WARPS * NSTAGE * stage_bytes<D>();
+  int cb, nch;
+  score_chunking(sh, &cb, &nch);
+  const int smem = NST * ScoreLayout<D>::STAGE;
   cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G>, (int)smem);
   if (e != cudaSuccess) return e;
-  score_kernel<D, G><<<grid, WARPS * 32, smem, s>>>(t, st, unit0, sh, q, sc, n_sealed, units);
+  score_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc, cb,
+                                                                      nch);
   return cudaGetLastError();
 }
 
