@@ -297,6 +297,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   const size_t o_err = take(sizeof(int));
   const size_t o_px = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
   const size_t o_cnt = take((size_t)c.batch * c.n_kv_heads * sizeof(int));
+  const size_t o_dcnt = take((size_t)c.batch * 2 * sizeof(int));
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     cudaGetLastError();
@@ -328,6 +329,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->sc.err = (int*)(bp + o_err);
   cc->sc.part_x = (float*)(bp + o_px);
   cc->sc.cnt = (int*)(bp + o_cnt);
+  cc->sc.dcnt = (int*)(bp + o_dcnt);
   cc->sc.ls = ls;
   cc->sc.max_chunks = (int)max_chunks;
 

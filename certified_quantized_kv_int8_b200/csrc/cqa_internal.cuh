@@ -86,6 +86,7 @@ struct Scratch {
   int* err;          // device error word (bit 0: a bounded wait gave up)
   float* part_x;     // [B*Hkv][max_chunks][G][3]  naive pass: (max Delta, residual m, residual l)
   int* cnt;          // [B*Hkv] naive pass: CTAs of the unit that have finished (0 between calls)
+  int* dcnt;         // [B][2] rank check: rung-3 heads, heads done (0 between calls)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
 };

@@ -28,68 +28,126 @@ struct KI {
 // (key descending, index ascending): true when a comes before b
 __device__ __forceinline__ bool before(KI a, KI b) { return a.k > b.k || (a.k == b.k && a.i < b.i); }
 
-// Best promoted block strictly after `prev` in the ranking order (warp-wide).
-__device__ KI next_best(const float* key, const uint8_t* bf, int nb, KI prev, int lane) {
-  KI best{-INFINITY, 0x7fffffff};
-  for (int j = lane; j < nb; j += 32) {
-    if (!(bf[j] & BF_KEY)) continue;
-    const KI c{key[j], j};
-    if (before(prev, c) && before(c, best)) best = c;
-  }
+// Rank check and the rung 3 / rung 4 decision, before the attention pass.
+// One CTA of DT threads per (batch row, query head).  The head's INT8 and FP16
+// block log-masses and the block flags are staged in shared memory when they
+// fit (else read in place); the ordered top-r lists are then built one rank
+// at a time by a CTA-wide arg-best under the (key desc, index asc) order.  The
+// last CTA of a batch row to finish takes the whole-layer decision (rung 4).
+constexpr int DT = 256;
+constexpr int DW = DT / 32;
+
+__device__ __forceinline__ KI ki_best(KI a, KI b) { return before(b, a) ? b : a; }
+
+__device__ __forceinline__ KI warp_best(KI v) {
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) {
     KI o;
-    o.k = __shfl_xor_sync(0xffffffffu, best.k, m);
-    o.i = __shfl_xor_sync(0xffffffffu, best.i, m);
-    if (before(o, best)) best = o;
+    o.k = __shfl_xor_sync(0xffffffffu, v.k, m);
+    o.i = __shfl_xor_sync(0xffffffffu, v.i, m);
+    v = ki_best(v, o);
   }
-  return best;
+  return v;
 }
 
-// Rank check and the rung 3 / rung 4 decision, before the attention pass.
-// grid B, one warp per query head (looping when n_q_heads > 32).
-__global__ void decide_kernel(DecodeShape sh, cqa_thresholds th, int need_dense, Scratch sc) {
-  __shared__ int n3;
-  extern __shared__ uint8_t r3[];  // [Hq]
-  const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
-  const bool naive = th.naive != 0;
-  if (threadIdx.x == 0) n3 = 0;
-  __syncthreads();
-  for (int h = warp; h < sh.Hq; h += nwarp) {
-    const int g = h / sh.G;
-    const int unit = b * sh.Hkv + g;
-    const size_t row = (size_t)b * sh.Hq + h;
-    uint8_t hf = sc.hflags[row];
-    if (!naive) {
-      const uint8_t* bf = sc.bflags + (size_t)unit * sh.nbm;
-      const float* e8 = sc.ell8 + row * sh.nbm;
-      const float* e16 = sc.ell16 + row * sh.nbm;
-      int np = 0;
-      for (int j = lane; j < sh.nb; j += 32) np += (bf[j] & BF_KEY) ? 1 : 0;
+__global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_thresholds th,
+                                                    int need_dense, Scratch sc, int staged) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ KI red[2][DW];
+  __shared__ int cnt[DW];
+  __shared__ int flag;
+  const int row_i = blockIdx.x;  // b * Hq + h
+  const int b = row_i / sh.Hq, h = row_i - b * sh.Hq;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int unit = b * sh.Hkv + h / sh.G;
+  const size_t row = (size_t)row_i;
+  const int nb = sh.nb;
+  const uint8_t* bf_g = sc.bflags + (size_t)unit * sh.nbm;
+  const float* e8_g = sc.ell8 + row * sh.nbm;
+  const float* e16_g = sc.ell16 + row * sh.nbm;
+  const float* e8 = e8_g;
+  const float* e16 = e16_g;
+  const uint8_t* bf = bf_g;
+  if (staged) {
+    float* s8 = reinterpret_cast<float*>(dsm);
+    float* s16 = s8 + nb;
+    uint8_t* sb = reinterpret_cast<uint8_t*>(s16 + nb);
+    for (int j = tid; j < nb; j += DT) {
+      s8[j] = e8_g[j];
+      s16[j] = e16_g[j];
+      sb[j] = bf_g[j];
+    }
+    e8 = s8;
+    e16 = s16;
+    bf = sb;
+    __syncthreads();
+  }
+  // promoted-block count
+  int np = 0;
+  for (int j = tid; j < nb; j += DT) np += (bf[j] & BF_KEY) ? 1 : 0;
 #pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) np += __shfl_xor_sync(0xffffffffu, np, m);
-      const int r = min(th.rank_r, np);
-      KI p8{INFINITY, -1}, p16{INFINITY, -1};
-      bool fail = false;
-      for (int k = 0; k < r && !fail; ++k) {
-        p8 = next_best(e8, bf, sh.nb, p8, lane);
-        p16 = next_best(e16, bf, sh.nb, p16, lane);
-        fail = p8.i != p16.i;
-      }
-      if (fail) hf |= HF_RANKFAIL;
+  for (int m = 16; m >= 1; m >>= 1) np += __shfl_xor_sync(0xffffffffu, np, m);
+  if (lane == 0) cnt[warp] = np;
+  __syncthreads();
+  np = 0;
+#pragma unroll
+  for (int w = 0; w < DW; ++w) np += cnt[w];
+  const int r = min(th.rank_r, np);
+  KI p8{INFINITY, -1}, p16{INFINITY, -1};
+  bool fail = false;
+  for (int k = 0; k < r && !fail; ++k) {
+    KI c8{-INFINITY, 0x7fffffff}, c16{-INFINITY, 0x7fffffff};
+    for (int j = tid; j < nb; j += DT) {
+      if (!(bf[j] & BF_KEY)) continue;
+      const KI a{e8[j], j}, a2{e16[j], j};
+      if (before(p8, a) && before(a, c8)) c8 = a;
+      if (before(p16, a2) && before(a2, c16)) c16 = a2;
     }
-    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
+    c8 = warp_best(c8);
+    c16 = warp_best(c16);
+    __syncthreads();  // the previous round's reads of red are done
     if (lane == 0) {
-      sc.hflags[row] = hf;
-      r3[h] = is3 ? 1 : 0;
-      if (is3) atomicAdd(&n3, 1);
+      red[0][warp] = c8;
+      red[1][warp] = c16;
     }
+    __syncthreads();
+    c8 = red[0][0];
+    c16 = red[1][0];
+#pragma unroll
+    for (int w = 1; w < DW; ++w) {
+      c8 = ki_best(c8, red[0][w]);
+      c16 = ki_best(c16, red[1][w]);
+    }
+    p8 = c8;
+    p16 = c16;
+    fail = p8.i != p16.i;  // the same on every thread
+  }
+  const bool naive = th.naive != 0;
+  if (tid == 0) {
+    uint8_t hf = sc.hflags[row];
+    if (!naive && fail) hf |= HF_RANKFAIL;
+    sc.hflags[row] = hf;
+    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
+    if (is3) atomicAdd(&sc.dcnt[2 * b], 1);
+    __threadfence();
+    flag = atomicAdd(&sc.dcnt[2 * b + 1], 1) == sh.Hq - 1;
   }
   __syncthreads();
+  if (!flag) return;
+  // the last head of the batch row: rung 3 per head, or rung 4 for the layer
+  __threadfence();
+  const int n3 = atomicAdd(&sc.dcnt[2 * b], 0);
   const bool layer = !naive && n3 >= need_dense;
-  for (int h = threadIdx.x; h < sh.Hq; h += blockDim.x)
-    sc.dense[(size_t)b * sh.Hq + h] = layer ? 4 : (r3[h] ? 3 : 0);
+  for (int hh = tid; hh < sh.Hq; hh += DT) {
+    const size_t rw = (size_t)b * sh.Hq + hh;
+    const uint8_t hf = __ldcg(&sc.hflags[rw]);
+    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
+    sc.dense[rw] = layer ? 4 : (is3 ? 3 : 0);
+  }
+  if (tid == 0) {
+    sc.dcnt[2 * b] = 0;
+    sc.dcnt[2 * b + 1] = 0;
+  }
 }
 
 __device__ __forceinline__ float cwarp_max(float x) {
@@ -270,8 +328,15 @@ cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, cons
 
 cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
                           const Scratch& sc, cudaStream_t s) {
-  const int threads = 32 * (sh.Hq < 32 ? sh.Hq : 32);
-  decide_kernel<<<sh.B, threads, sh.Hq, s>>>(sh, th, need_dense, sc);
+  // stage the head's keys and flags in shared memory up to 96 KiB
+  const size_t bytes = (size_t)sh.nb * 9;
+  const int staged = bytes <= 96u * 1024u ? 1 : 0;
+  const int smem = staged ? (int)((bytes + 15) / 16 * 16) : 0;
+  if (smem > 48 * 1024) {
+    cudaError_t e = ensure_dynamic_smem((const void*)decide_kernel, smem);
+    if (e != cudaSuccess) return e;
+  }
+  decide_kernel<<<sh.B * sh.Hq, DT, smem, s>>>(sh, th, need_dense, sc, staged);
   return cudaGetLastError();
 }
 

@@ -153,21 +153,23 @@ __device__ double naive_e_key(double dT, double dA, double m8T) {
   return fmin(tanh(0.5 * dT), m_ub * expm1(2.0 * dT));
 }
 
-// Arrival of one CTA of a (batch row, kv head) unit; the last of its nparts
-// CTAs merges the unit's partials (split-K combine) into the outputs: the
+// Arrival of one CTA of a (batch row, kv head) unit; the last of its narr
+// CTAs merges the unit's nparts partials (split-K combine; the last part is
+// the residual block's) into the outputs: the
 // outputs o / L, E_key from the largest Delta and the residual's mass, and
 // E_val = sum of eta-weighted mass / L.  Every CTA of the launch calls this
 // exactly once, also after a failed wait, so the arrival counter returns to
 // zero for the next launch.
 template <int D, int G>
-__device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int nparts, int unit,
+__device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int nparts, int narr,
+                                   int unit,
                                    size_t hrow0, float* __restrict__ out,
                                    float* __restrict__ e_key, float* __restrict__ e_val,
                                    uint8_t* __restrict__ rung, float* wsm, int* flag) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   __threadfence();  // this thread's partials, before the arrival below
   __syncthreads();
-  if (tid == 0) *flag = atomicAdd(&sc.cnt[unit], 1) == nparts - 1;
+  if (tid == 0) *flag = atomicAdd(&sc.cnt[unit], 1) == narr - 1;
   __syncthreads();
   if (!*flag) return;
   __threadfence();
@@ -296,7 +298,7 @@ __device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int
 template <int D, int G>
 __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     naive_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
-                 Scratch sc, int chunk_blocks, int nres_chunk, int trace,
+                 Scratch sc, int trace,
                  float* __restrict__ out, float* __restrict__ e_key, float* __restrict__ e_val,
                  uint8_t* __restrict__ rung) {
   using LY = NaiveLayout<D>;
@@ -332,77 +334,16 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
   }
   if (tid < G) S.dmax[tid] = 0.f;  // published by the barrier before the first block
 
-  // ---- the exact residual block: a CTA of its own (the last chunk index) ----
-  if (chunk == nres_chunk) {
-    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK] base-2 logits, then weights
-    float* mst = lg + G * BLK;                  // [G][2]
-    const int r = sh.r;
-    __syncthreads();
-    const __half* kr = t.kres + u * st.res;
-    const __half* vr = t.vres + u * st.res;
-    constexpr int CPL = D / 32;
-    for (int tt = warp; tt < r; tt += NW) {
-      float kf[CPL];
-#pragma unroll
-      for (int i = 0; i < CPL; i += 2) {
-        const float2 f = __half22float2(
-            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
-        kf[i] = f.x;
-        kf[i + 1] = f.y;
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = 0.f;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
-        v = nwarp_sum(v);
-        if (lane == 0) lg[h * BLK + tt] = v;
-      }
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += NW) {
-      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
-      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
-      const float m = nwarp_max(fmaxf(x0, x1));
-      const float e0 = lane < r ? exp2f(x0 - m) : 0.f;
-      const float e1 = lane + 32 < r ? exp2f(x1 - m) : 0.f;
-      const float l = nwarp_sum(e0 + e1);
-      lg[h * BLK + lane] = e0;
-      lg[h * BLK + lane + 32] = e1;
-      if (lane == 0) {
-        mst[2 * h] = r > 0 ? m * LN2 : -INFINITY;
-        mst[2 * h + 1] = l;
-        sc.ell_res[hrow0 + h] = r > 0 ? (m + log2f(l)) * LN2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-    for (int c = tid; c < D; c += NT) {
-      float o[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) o[h] = 0.f;
-      for (int tt = 0; tt < r; ++tt) {
-        const float v = __half2float(vr[(size_t)tt * D + c]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) o[h] = fmaf(lg[h * BLK + tt], v, o[h]);
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) sc.part_o[(pbase + h) * D + c] = o[h];
-    }
-    if (tid < G) {
-      sc.part_s[(pbase + tid) * 3 + 0] = mst[2 * tid];
-      sc.part_s[(pbase + tid) * 3 + 1] = mst[2 * tid + 1];
-      sc.part_s[(pbase + tid) * 3 + 2] = 0.f;
-      sc.part_x[(pbase + tid) * 3 + 0] = 0.f;
-      sc.part_x[(pbase + tid) * 3 + 1] = mst[2 * tid];
-      sc.part_x[(pbase + tid) * 3 + 2] = mst[2 * tid + 1];
-    }
-    naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
-                             reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::RES, &S.last);
-    return;
-  }
-
-  const int j0 = chunk * chunk_blocks;
-  const int nblk = max(0, min(sh.nb, j0 + chunk_blocks) - j0);
+  // work items: the nb sealed blocks, then the residual block (item nb); the
+  // nch CTAs of a unit take floor or ceil((nb + 1) / nch) consecutive items
+  const int nch = gridDim.x;
+  const int items = sh.nb + 1;
+  const int base = items / nch, rem = items - base * nch;
+  const int i0 = chunk * base + min(chunk, rem);
+  const int i1 = i0 + base + (chunk < rem ? 1 : 0);
+  const int j0 = i0;
+  const int nblk = max(0, min(i1, sh.nb) - i0);
+  const bool do_res = i1 > sh.nb;  // the unit's last CTA
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) mbar_init(&S.bar[s], 1);
     mbar_init_fence();
@@ -646,7 +587,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       for (int k2 = k; k2 <= hi; ++k2)
         mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
     }
-    naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
+    naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, hrow0, out, e_key, e_val, rung,
                              reinterpret_cast<float*>(dsm), &S.last);
     return;
   }
@@ -732,29 +673,92 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     sc.part_x[(pbase + tid) * 3 + 1] = -INFINITY;
     sc.part_x[(pbase + tid) * 3 + 2] = 0.f;
   }
-  naive_arrive_merge<D, G>(sh, sc, nres_chunk + 1, unit, hrow0, out, e_key, e_val, rung,
-                           reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::MAIN, &S.last);
+  // ---- the exact residual block (item nb), by the unit's last CTA, into partial slot nch ----
+  if (do_res) {
+    __syncthreads();  // the warps' states above are read: the stage area is free
+    const size_t rbase = ((size_t)unit * sc.max_chunks + nch) * G;
+    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK] base-2 logits, then weights
+    float* mst = lg + G * BLK;                  // [G][2]
+    const int r = sh.r;
+    const __half* kr = t.kres + u * st.res;
+    const __half* vr = t.vres + u * st.res;
+    constexpr int CPL = D / 32;
+    for (int tt = warp; tt < r; tt += NW) {
+      float kf[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; i += 2) {
+        const float2 f = __half22float2(
+            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
+        kf[i] = f.x;
+        kf[i + 1] = f.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
+        v = nwarp_sum(v);
+        if (lane == 0) lg[h * BLK + tt] = v;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += NW) {
+      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
+      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
+      const float m = nwarp_max(fmaxf(x0, x1));
+      const float e0 = lane < r ? exp2f(x0 - m) : 0.f;
+      const float e1 = lane + 32 < r ? exp2f(x1 - m) : 0.f;
+      const float l = nwarp_sum(e0 + e1);
+      lg[h * BLK + lane] = e0;
+      lg[h * BLK + lane + 32] = e1;
+      if (lane == 0) {
+        mst[2 * h] = r > 0 ? m * LN2 : -INFINITY;
+        mst[2 * h + 1] = l;
+        sc.ell_res[hrow0 + h] = r > 0 ? (m + log2f(l)) * LN2 : -INFINITY;
+      }
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += NT) {
+      float o[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) o[h] = 0.f;
+      for (int tt = 0; tt < r; ++tt) {
+        const float v = __half2float(vr[(size_t)tt * D + c]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = fmaf(lg[h * BLK + tt], v, o[h]);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) sc.part_o[(rbase + h) * D + c] = o[h];
+    }
+    if (tid < G) {
+      sc.part_s[(rbase + tid) * 3 + 0] = mst[2 * tid];
+      sc.part_s[(rbase + tid) * 3 + 1] = mst[2 * tid + 1];
+      sc.part_s[(rbase + tid) * 3 + 2] = 0.f;
+      sc.part_x[(rbase + tid) * 3 + 0] = 0.f;
+      sc.part_x[(rbase + tid) * 3 + 1] = mst[2 * tid];
+      sc.part_x[(rbase + tid) * 3 + 2] = mst[2 * tid + 1];
+    }
+  }
+  naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, hrow0, out, e_key, e_val, rung,
+                           reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::AT, &S.last);
 }
 
-// chunking of the streaming pass: about four resident CTAs per SM over all units
-void naive_chunking(const DecodeShape& sh, int max_chunks, int* cb, int* nch) {
+// CTAs per unit of the streaming pass: four resident CTAs per SM hold the
+// whole grid (one wave), so the unit's last arrival is never a CTA that
+// waited for a free slot
+int naive_chunks(const DecodeShape& sh, int max_chunks) {
   const int units = sh.B * sh.Hkv;
-  int per_unit = (148 * 4 + units - 1) / units;
+  int per_unit = 148 * 4 / units;
   if (per_unit > max_chunks - 1) per_unit = max_chunks - 1;  // one partial slot for the residual
-  if (per_unit < 1) per_unit = 1;
-  int c = sh.nb > 0 ? (sh.nb + per_unit - 1) / per_unit : 1;
-  if (c < 1) c = 1;
-  int n = sh.nb > 0 ? (sh.nb + c - 1) / c : 1;
-  *cb = c;
-  *nch = n < 1 ? 1 : n;
+  if (per_unit > sh.nb + 1) per_unit = sh.nb + 1;
+  return per_unit < 1 ? 1 : per_unit;
 }
 
 template <int D, int G>
 cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                     const __half* q, const Scratch& sc, float* out, float* e_key, float* e_val,
                     uint8_t* rung, int trace, cudaStream_t s) {
-  int cb, nch;
-  naive_chunking(sh, sc.max_chunks, &cb, &nch);
+  const int nch = naive_chunks(sh, sc.max_chunks);
   const int smem = NST * NaiveLayout<D>::STAGE;
   // the merge keeps (nch + 1) * G weights, G inverse sums and NT float4 partial
   // sums in the stage area, after what the CTAs still hold there
@@ -763,8 +767,8 @@ cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeSh
   if (merge_floats * 4 > (size_t)smem) return cudaErrorInvalidValue;
   cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G>, (int)smem);
   if (e != cudaSuccess) return e;
-  naive_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(
-      t, st, unit0, sh, q, sc, cb, nch, trace, out, e_key, e_val, rung);
+  naive_kernel<D, G><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(
+      t, st, unit0, sh, q, sc, trace, out, e_key, e_val, rung);
   return cudaGetLastError();
 }
 

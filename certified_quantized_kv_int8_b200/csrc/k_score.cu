@@ -95,7 +95,7 @@ struct ScoreSmem {
 template <int D, int G>
 __global__ void __launch_bounds__(NT, 5)
     score_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
-                 Scratch sc, int chunk_blocks, int nres_chunk) {
+                 Scratch sc) {
   using LY = ScoreLayout<D>;
   constexpr int CPT = D / CH;     // lanes per token row
   constexpr int RPW = 32 / CPT;   // rows per warp instruction
@@ -120,52 +120,16 @@ __global__ void __launch_bounds__(NT, 5)
     S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * sh.sigma;
   }
 
-  // ---- the residual block: exact logits from the FP16 keys in device memory ----
-  if (chunk == nres_chunk) {
-    __syncthreads();
-    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK]
-    const int r = sh.r;
-    const __half* kr = t.kres + u * st.res;
-    constexpr int CPL = D / 32;
-    for (int tt = warp; tt < r; tt += NW) {
-      float kf[CPL];
-#pragma unroll
-      for (int i = 0; i < CPL; i += 2) {
-        const float2 f = __half22float2(
-            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
-        kf[i] = f.x;
-        kf[i + 1] = f.y;
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = 0.f;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
-        v = swarp_sum(v);
-        if (lane == 0) lg[h * BLK + tt] = v;
-      }
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += NW) {
-      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
-      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
-      float* lo = sc.logits + (hrow0 + h) * sc.ls + (size_t)sh.nb * BLK;
-      if (lane < r) lo[lane] = x0;
-      if (lane + 32 < r) lo[lane + 32] = x1;
-      float lse = -INFINITY;
-      if (r > 0) {
-        const float m = swarp_max(fmaxf(x0, x1));
-        const float ssum = swarp_sum((lane < r ? expf(x0 - m) : 0.f) +
-                                     (lane + 32 < r ? expf(x1 - m) : 0.f));
-        lse = m + logf(ssum);
-      }
-      if (lane == 0) sc.ell_res[hrow0 + h] = lse;
-    }
-    return;
-  }
-
-  const int j0 = chunk * chunk_blocks;
-  const int nblk = max(0, min(sh.nb, j0 + chunk_blocks) - j0);
+  // work items: the nb sealed blocks, then the residual block (item nb); the
+  // CTAs of a unit take floor or ceil((nb + 1) / gridDim.x) consecutive items
+  const int nch = gridDim.x;
+  const int items = sh.nb + 1;
+  const int base = items / nch, rem = items - base * nch;
+  const int i0 = chunk * base + min(chunk, rem);
+  const int i1 = i0 + base + (chunk < rem ? 1 : 0);
+  const int j0 = i0;
+  const int nblk = max(0, min(i1, sh.nb) - i0);
+  const bool do_res = i1 > sh.nb;  // the unit's last CTA
   if (tid == 0) {
     for (int s2 = 0; s2 < NST; ++s2) mbar_init(&S.bar[s2], 1);
     mbar_init_fence();
@@ -328,31 +292,67 @@ __global__ void __launch_bounds__(NT, 5)
     return;
   }
   if (nblk > 0) finish_ell((nblk - 1) & 1, j0 + nblk - 1);
+
+  // ---- the residual block (item nb), by the unit's last CTA: exact logits from
+  // the FP16 keys in device memory ----
+  if (do_res) {
+    float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK]
+    const int r = sh.r;
+    const __half* kr = t.kres + u * st.res;
+    constexpr int CPL = D / 32;
+    for (int tt = warp; tt < r; tt += NW) {
+      float kf[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; i += 2) {
+        const float2 f = __half22float2(
+            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
+        kf[i] = f.x;
+        kf[i + 1] = f.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
+        v = swarp_sum(v);
+        if (lane == 0) lg[h * BLK + tt] = v;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += NW) {
+      const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
+      const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
+      float* lo = sc.logits + (hrow0 + h) * sc.ls + (size_t)sh.nb * BLK;
+      if (lane < r) lo[lane] = x0;
+      if (lane + 32 < r) lo[lane + 32] = x1;
+      float lse = -INFINITY;
+      if (r > 0) {
+        const float m = swarp_max(fmaxf(x0, x1));
+        const float ssum = swarp_sum((lane < r ? expf(x0 - m) : 0.f) +
+                                     (lane + 32 < r ? expf(x1 - m) : 0.f));
+        lse = m + logf(ssum);
+      }
+      if (lane == 0) sc.ell_res[hrow0 + h] = lse;
+    }
+  }
 }
 
-// chunking: about five resident CTAs per SM over all units, one more per unit
-// for the residual block
-void score_chunking(const DecodeShape& sh, int* cb, int* nch) {
+// CTAs per unit: five resident CTAs per SM hold the whole grid (one wave)
+int score_chunks(const DecodeShape& sh) {
   const int units = sh.B * sh.Hkv;
-  int per_unit = (148 * 5 + units - 1) / units;
+  int per_unit = 148 * 5 / units;
   if (per_unit < 1) per_unit = 1;
-  int c = sh.nb > 0 ? (sh.nb + per_unit - 1) / per_unit : 1;
-  if (c < 1) c = 1;
-  const int n = sh.nb > 0 ? (sh.nb + c - 1) / c : 0;
-  *cb = c;
-  *nch = n;
+  return per_unit < sh.nb + 1 ? per_unit : sh.nb + 1;
 }
 
 template <int D, int G>
 cudaError_t launch_score_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                            const __half* q, const Scratch& sc, cudaStream_t s) {
-  int cb, nch;
-  score_chunking(sh, &cb, &nch);
+  const int nch = score_chunks(sh);
   const int smem = NST * ScoreLayout<D>::STAGE;
   cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G>, (int)smem);
   if (e != cudaSuccess) return e;
-  score_kernel<D, G><<<dim3(nch + 1, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc, cb,
-                                                                      nch);
+  score_kernel<D, G><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc);
   return cudaGetLastError();
 }
 
