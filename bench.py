@@ -454,6 +454,9 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
                                          "hbm": dp["hbm_bytes"]},
         "traffic": (rec["dram_bytes_per_block"] * census["blocks_per_layer"] if rec else None),
     }
+    if dp["bound"] == "h2d" and phase_n.get("prefetch"):
+        roofline["note"] = ("the link is shared with the copy-engine key prefetch running beside "
+                            "this kernel; step_roofline has the link over the whole step")
     # the host link over the whole certified step: key copies by the copy engine
     # plus every kernel's host-link reads, against the pinned-copy rate
     link_bytes = sum(p["host_link_bytes"] * p["launches"] for p in phases.values()) / args.steps

@@ -66,10 +66,13 @@ def test_decode_tiny(cqa, case, ctx):
 
 
 @pytest.mark.parametrize("ctx", [1, 37, 64, 65, 128 + 63])
-def test_decode_short_contexts(cqa, ctx):
+@pytest.mark.parametrize("naive", [False, True])
+def test_decode_short_contexts(cqa, ctx, naive):
+    """No sealed block, one, two: the streaming passes then run fewer CTAs per unit
+    than their grid target, down to one that holds only the residual block."""
     w = sk.WORKLOADS["tiny"]
-    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.7})
-    _check(cqa, w, ctx, th, label=f"ctx{ctx}")
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.7, "naive": naive})
+    _check(cqa, w, ctx, th, label=f"ctx{ctx}{' naive' if naive else ''}")
 
 
 def test_decode_llama8b_8k(cqa):
