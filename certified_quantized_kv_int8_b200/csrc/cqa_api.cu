@@ -659,7 +659,14 @@ int cqa_device_status(cqa_cache* cc, int32_t* status) {
   if (cudaDeviceSynchronize() != cudaSuccess) return CQA_ERR_CUDA;
   if (cudaMemcpy(&v, cc->sc.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return CQA_ERR_CUDA;
-  if (v && cudaMemset(cc->sc.err, 0, sizeof(int)) != cudaSuccess) return CQA_ERR_CUDA;
+  if (v) {
+    // a kernel that gave up may have left its arrival counters short of zero
+    const size_t units = (size_t)cc->cfg.batch * cc->cfg.n_kv_heads;
+    if (cudaMemset(cc->sc.err, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(cc->sc.cnt, 0, units * sizeof(int)) != cudaSuccess ||
+        cudaMemset(cc->sc.dcnt, 0, (size_t)cc->cfg.batch * 2 * sizeof(int)) != cudaSuccess)
+      return CQA_ERR_CUDA;
+  }
   *status = v;
   return CQA_OK;
 }

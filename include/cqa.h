@@ -177,8 +177,9 @@ int64_t cqa_debug_export(cqa_cache* cache, int layer, int what, void* host_dst, 
 /* Device status word of the cache's kernels, read after synchronising the
  * device and then cleared.  The streaming kernels wait for their own bulk
  * copies with a bounded number of polls; a wait that runs out sets bit 0
- * (and that kernel's results are not valid).  *status = 0 means every kernel
- * since the last call completed normally. */
+ * (and that kernel's results are not valid).
+ * *status = 0 means every kernel since the last call completed normally.  A
+ * nonzero status also resets the kernels' arrival counters. */
 int cqa_device_status(cqa_cache* cache, int32_t* status);
 
 /* Self-test of the failure path above: launches one kernel that waits, for at
