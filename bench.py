@@ -255,6 +255,33 @@ def phase_bytes(c: dict, w: sk.Workload, staged_frac: float = 0.0) -> dict:
     }
 
 
+def accuracy_on_layer(cache, layer, q, thr_list, dense):
+    """Max-abs error against exact attention and the certified bound per threshold set
+    (untimed).  The bound is R_V * E_key + E_val per head, R_V = max_c (vmax_c - vmin_c)
+    of the head's kv head (Methodology §2)."""
+    B, Hq, Hkv = cache.batch, cache.n_q_heads, cache.n_kv_heads
+    vr = torch.from_numpy(cache.export(layer, 5)).double()  # [B][Hkv][2][d]
+    r_v = (vr[:, :, 1] - vr[:, :, 0]).amax(dim=-1)          # [B][Hkv]
+    r_v = r_v.repeat_interleave(Hq // Hkv, dim=1)           # [B][Hq]
+    rows = []
+    for thr in thr_list:
+        trace = cache.alloc_trace(layer)
+        o, ek, ev, rg = cache.decode(layer, q, thr, trace=trace)
+        torch.cuda.synchronize()
+        err = (o.double() - dense.double()).abs().amax(dim=-1).cpu()  # [B][Hq]
+        bound = r_v * ek.double().cpu() + ev.double().cpu()
+        bf = trace["block_flags"]
+        rows.append({
+            "max_abs_err": float(err.max()),
+            "max_bound": float(bound.max()),
+            "bound_holds": bool((err <= bound * (1 + 1e-3) + 1e-5).all()),  # + fp32 noise
+            "value_promoted_frac": float(((bf & 2) != 0).float().mean()),
+            "max_e_val": float(ev.max()),
+            "rung_histogram": [int((rg == k).sum()) for k in range(5)],
+        })
+    return rows
+
+
 # --------------------------------------------------------------- our arm ----
 
 def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | None:
@@ -412,6 +439,36 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     n_el, _ = timed(first, n_naive, th_naive, label="int8_int4")
     n_max = max_over_ranks(n_el, dist, device)
     _, nprof = timed(first + n_naive, n_naive, th_naive, profile=True, label="int8_int4_profiled")
+
+    # accuracy against exact attention on one layer (untimed): the certified path
+    # against the INT8/INT4 path; on the needle workload the layer with ties planted
+    # in every kv group
+    acc_layer = min(w.tie_layer_all, L - 1) if w.needle else 0
+    q_acc = inputs[first + 2 * n_naive - 1][0][acc_layer]
+    dense = cache.dense_reference(acc_layer, q_acc)
+    a_c, a_n = accuracy_on_layer(cache, acc_layer, q_acc, [th, th_naive], dense)
+    accuracy = {"layer": acc_layer, "certified": a_c, "int8_int4": a_n}
+    vtol_sweep = None
+    if args.vtol_sweep:
+        # the value-side ablation: value promotion from none to every block (all FP16 values)
+        # on layer 0 (on the needle workload layer 17 goes whole-layer dense at any v_tol)
+        q0 = inputs[first + 2 * n_naive - 1][0][0]
+        dense0 = cache.dense_reference(0, q0)
+        tols = [float("inf"), th.v_tol, th.v_tol / 10, th.v_tol / 100, 0.0]
+        thrs = [dataclasses.replace(th, v_tol=v) for v in tols]
+        rows = accuracy_on_layer(cache, 0, q0, thrs, dense0)
+        for v, thr, row in zip(tols, thrs, rows):
+            torch.cuda.synchronize(device)
+            ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ta.record(stream)
+            for _ in range(5):
+                cache.decode(0, q0, thr, outputs=outs, stream=stream)
+            tb.record(stream)
+            torch.cuda.synchronize(device)
+            row["layer"] = 0
+            row["v_tol"] = v if v != float("inf") else "inf"
+            row["decode_ms"] = ta.elapsed_time(tb) / 5
+        vtol_sweep = rows
     nb_total = sum(cache.length(layer) // BLOCK for layer in range(L))
     t1_bytes = nb_total * B * Hkv * tier1_bytes_per_block(d)  # per step (lengths at the end)
     peaks = measured_peaks()
@@ -545,12 +602,15 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "prefetch_copy_gbs": phases.get("prefetch", {}).get("achieved_gbs"),
             "rung_histogram": census["rungs"],
         },
+        "accuracy": accuracy,
         "phases": phases,
         "gpu_launches": int(sum(v for k, v in phase_n.items() if k != "prefetch")),
         "clocks": clk,
     }
     if e2e:
         res["e2e"] = e2e
+    if vtol_sweep:
+        res["vtol_sweep"] = vtol_sweep
     cache.close()
     return res
 
@@ -649,6 +709,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(sk.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--vtol-sweep", action="store_true",
+                    help="add the value-side ablation: one layer decoded at v_tol = inf, the "
+                         "default, /10, /100 and 0 (every block's FP16 values)")
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only the first N layers (profiling captures; the reported "
                          "line then covers N layers, not the workload's step)")
