@@ -82,6 +82,66 @@ struct Group {
   __device__ void sync() const { group_bar(id, nthreads); }
 };
 
+// Bitonic sort (ascending) of one head's keys by its GT-thread group, E keys per
+// thread in registers: thread tg holds positions tg*E .. tg*E + E - 1.  Distances
+// below E are swaps inside a thread, below 32*E shuffles inside a warp; only the
+// widest stages exchange through shared memory (x, E*GT keys, laid out [r][tg] so
+// a warp's accesses are consecutive).  On entry keys[0, E*GT) holds the keys; on
+// exit it holds them sorted.
+template <int E>
+__device__ void group_sort(uint64_t* keys, int tg, int GT, const Group& grp) {
+  uint64_t v[E];
+#pragma unroll
+  for (int r = 0; r < E; ++r) v[r] = keys[tg * E + r];
+  grp.sync();  // every thread has its keys: the array is free for the exchanges
+  const int n = GT * E;
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+#pragma unroll
+        for (int jj = E / 2; jj >= 1; jj >>= 1) {
+          if (jj == j) {
+#pragma unroll
+            for (int r = 0; r < E; ++r) {
+              if ((r & jj) == 0) {
+                const bool up = ((tg * E + r) & k) == 0;
+                const uint64_t a = v[r], b = v[r + jj];
+                if ((a > b) == up) {
+                  v[r] = b;
+                  v[r + jj] = a;
+                }
+              }
+            }
+          }
+        }
+      } else {
+        const int m = j / E;  // distance in threads
+        const bool keep_min = ((tg & m) == 0) == (((tg * E) & k) == 0);
+        if (m < 32) {
+#pragma unroll
+          for (int r = 0; r < E; ++r) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, v[r], m);
+            v[r] = keep_min ? (o < v[r] ? o : v[r]) : (o > v[r] ? o : v[r]);
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < E; ++r) keys[r * GT + tg] = v[r];
+          grp.sync();
+#pragma unroll
+          for (int r = 0; r < E; ++r) {
+            const uint64_t o = keys[r * GT + (tg ^ m)];
+            v[r] = keep_min ? (o < v[r] ? o : v[r]) : (o > v[r] ? o : v[r]);
+          }
+          grp.sync();
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < E; ++r) keys[tg * E + r] = v[r];
+  grp.sync();
+}
+
 __device__ double e_key_bound(double dT, double dA, double m8T) {
   const double a = m8T * exp(dT);
   const double m_ub = a > 0.0 ? a / (a + (1.0 - m8T) * exp(-dA)) : 0.0;
@@ -156,8 +216,18 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
   grp.sync();
 
   // ---- bitonic sort of this head's NP keys ----
+  // NP keys padded with sentinels to E = NP / GT >= 1 keys per thread (registers,
+  // up to 8 within the 64 registers a thread has at 1024 threads per CTA)
+  const int Ek = NP > GT ? NP / GT : 1;
+  switch (Ek) {
+    case 1: group_sort<1>(keys, tg, GT, grp); break;
+    case 2: group_sort<2>(keys, tg, GT, grp); break;
+    case 4: group_sort<4>(keys, tg, GT, grp); break;
+    case 8: group_sort<8>(keys, tg, GT, grp); break;
+    default: break;
+  }
   const int half = NP >> 1;
-  for (int k = 2; k <= NP; k <<= 1) {
+  for (int k = 2; Ek > 8 && k <= NP; k <<= 1) {  // longer heads: in shared memory
     for (int jj = k >> 1; jj > 0; jj >>= 1) {
       for (int p = tg; p < half; p += GT) {
         const int a = 2 * jj * (p / jj) + (p % jj);
@@ -287,6 +357,7 @@ cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const 
                             const cqa_thresholds& th, const Scratch& sc, cudaStream_t s) {
   int NP = 2;
   while (NP < sh.nb) NP <<= 1;
+  if (NP < THREADS / G) NP = THREADS / G;  // at least one key per thread of a head group
   const size_t smem = (size_t)G * NP * 8 + (size_t)G * sh.nb * 4 + 2 * (size_t)sh.nb;
   cudaError_t e = ensure_dynamic_smem((const void*)select_kernel<G>, (int)smem);
   if (e != cudaSuccess) return e;
@@ -299,6 +370,7 @@ cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const 
 size_t select_smem_bytes(int G, int nb) {
   int NP = 2;
   while (NP < nb) NP <<= 1;
+  if (NP < THREADS / G) NP = THREADS / G;
   return (size_t)G * NP * 8 + (size_t)G * nb * 4 + 2 * (size_t)nb;
 }
 
