@@ -38,6 +38,7 @@ cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
 struct cqa_cache {
   cqa_config cfg;
   int G, nbm;
+  int sms;             // streaming multiprocessors of the device
   Strides st;
   Tier1 t;
   Scratch sc;
@@ -82,10 +83,11 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-constexpr int kTargetCtas = 148 * 4;  // attend grid target: several waves over 148 SMs
+// attend grid target: four CTAs per SM
+int target_ctas(int sms) { return sms * 4; }
 
-void chunking(int units, int nb, int* chunk_blocks, int* nchunks) {
-  int per_unit = (kTargetCtas + units - 1) / units;
+void chunking(int units, int nb, int sms, int* chunk_blocks, int* nchunks) {
+  int per_unit = (target_ctas(sms) + units - 1) / units;
   if (per_unit < 1) per_unit = 1;
   int cb = nb > 0 ? (nb + per_unit - 1) / per_unit : 1;
   if (cb < 1) cb = 1;
@@ -94,7 +96,7 @@ void chunking(int units, int nb, int* chunk_blocks, int* nchunks) {
   *nchunks = nc < 1 ? 1 : nc;
 }
 
-int max_chunks_for(int units) { return (kTargetCtas + units - 1) / units + 1; }
+int max_chunks_for(int units, int sms) { return (target_ctas(sms) + units - 1) / units + 1; }
 
 DecodeShape shape_of(const cqa_cache* c, int T) {
   DecodeShape sh;
@@ -107,7 +109,8 @@ DecodeShape shape_of(const cqa_cache* c, int T) {
   sh.r = T - sh.nb * BLK;
   sh.nbm = c->nbm;
   sh.sigma = (float)(1.0 / sqrt((double)sh.d));
-  chunking(sh.B * sh.Hkv, sh.nb, &sh.chunk_blocks, &sh.nchunks);
+  sh.sms = c->sms;
+  chunking(sh.B * sh.Hkv, sh.nb, sh.sms, &sh.chunk_blocks, &sh.nchunks);
   return sh;
 }
 
@@ -263,7 +266,15 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->st = make_strides(nbm, d, c.max_ctx);
   const size_t units = (size_t)c.n_layers * c.batch * c.n_kv_heads;
   const size_t hq_rows = (size_t)c.batch * c.n_q_heads;
-  const size_t max_chunks = (size_t)max_chunks_for(c.batch * c.n_kv_heads);
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c.device) != cudaSuccess ||
+      sms < 1) {
+    cudaGetLastError();
+    delete cc;
+    return CQA_ERR_CUDA;
+  }
+  cc->sms = sms;
+  const size_t max_chunks = (size_t)max_chunks_for(c.batch * c.n_kv_heads, sms);
 
   // one device allocation, carved into aligned pieces
   size_t off = 0;

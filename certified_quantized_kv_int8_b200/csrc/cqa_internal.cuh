@@ -93,6 +93,7 @@ struct Scratch {
 
 struct DecodeShape {
   int B, Hq, Hkv, G, d, nb, r, nbm, nchunks, chunk_blocks;
+  int sms;  // streaming multiprocessors of the cache's device (grid sizing)
   float sigma;
 };
 

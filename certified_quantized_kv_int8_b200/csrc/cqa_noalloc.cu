@@ -256,7 +256,13 @@ extern "C" int cqa_dense_attention_noalloc(const void* q_fp16, const void* k_fp1
   const size_t per_part = (size_t)G * (head_dim + 3) * sizeof(float);
   const long long cap_parts = (long long)(CQA_NOALLOC_SCRATCH_BYTES / per_part);
   if (units > cap_parts) return CQA_ERR_CAPACITY;  // even one chunk per unit does not fit
-  long long per_unit = (148 * 4 + units - 1) / units;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();
+    return CQA_ERR_CUDA;
+  }
+  long long per_unit = ((long long)sms * 4 + units - 1) / units;
   if (per_unit > cap_parts / units) per_unit = cap_parts / units;
   if (per_unit < 1) per_unit = 1;
   const int chunk_blocks = (int)((nblk + per_unit - 1) / per_unit);
@@ -266,8 +272,7 @@ extern "C" int cqa_dense_attention_noalloc(const void* q_fp16, const void* k_fp1
 
   // one-time set-up per device: the host-side name of the array is not a
   // device address, so look the address up with this device current
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return CQA_ERR_CUDA;
+  if (dev < 0 || dev >= 256) return CQA_ERR_CUDA;
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);

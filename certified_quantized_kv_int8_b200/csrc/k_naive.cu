@@ -748,7 +748,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 // waited for a free slot
 int naive_chunks(const DecodeShape& sh, int max_chunks) {
   const int units = sh.B * sh.Hkv;
-  int per_unit = 148 * 4 / units;
+  int per_unit = sh.sms * 4 / units;
   if (per_unit > max_chunks - 1) per_unit = max_chunks - 1;  // one partial slot for the residual
   if (per_unit > sh.nb + 1) per_unit = sh.nb + 1;
   return per_unit < 1 ? 1 : per_unit;

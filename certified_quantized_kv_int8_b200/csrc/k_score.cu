@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(NT, 5)
 // CTAs per unit: five resident CTAs per SM hold the whole grid (one wave)
 int score_chunks(const DecodeShape& sh) {
   const int units = sh.B * sh.Hkv;
-  int per_unit = 148 * 5 / units;
+  int per_unit = sh.sms * 5 / units;
   if (per_unit < 1) per_unit = 1;
   return per_unit < sh.nb + 1 ? per_unit : sh.nb + 1;
 }
