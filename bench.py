@@ -656,9 +656,19 @@ def cpu_baseline(w: sk.Workload, th, budget_s: float = 20.0) -> dict:
         layer += 1
     per = statistics.mean(secs)
     step_s = per * w.n_layers * w.batch
-    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} of {w.n_layers * w.batch} (layer, batch row) decodes of one step, "
-                      f"{per:.2f} s each, scaled to the full step (appends not included)"}
+    res = {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{n} of {w.n_layers * w.batch} (layer, batch row) decodes of one step, "
+                     f"{per:.2f} s each, scaled to the full step (appends not included)"}
+    # the same oracle on one thread (one (layer, batch row) decode)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            s1, _ = oracle_sample_seconds(w, 0, 0, th)
+        res["single_thread_value"] = 1.0 / (s1 * w.n_layers * w.batch)
+        res["single_thread_sample"] = f"1 (layer, batch row) decode, {s1:.2f} s, scaled"
+    except ImportError:
+        pass
+    return res
 
 
 def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
@@ -703,7 +713,8 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=64,
+                    help="timed steps (64: the 32K workload's append-and-decode steps)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
