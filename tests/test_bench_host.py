@@ -60,3 +60,14 @@ def test_reference_arm_prints_one_line(capsys):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_reports_threads_and_single_thread():
+    """The oracle timing beside the GPU numbers: its BLAS threads, and one thread."""
+    import certified_quantized_kv_int8_b200 as cqa
+    import synthetic_kv as sk
+    w = sk.WORKLOADS["tiny"]
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    d = bench.cpu_baseline(w, th, budget_s=1.0)
+    assert d["kind"] == "oracle" and d["value"] > 0 and d["cores"] >= 1
+    assert d["single_thread_value"] > 0
