@@ -674,7 +674,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     sc.part_x[(pbase + tid) * 3 + 1] = -INFINITY;
     sc.part_x[(pbase + tid) * 3 + 2] = 0.f;
   }
-  // ---- the exact residual block (item nb), by the unit's last CTA, into partial slot nch ----
+  // ---- the exact residual block (item nb), by the CTA holding it, into partial slot nch ----
   if (do_res) {
     __syncthreads();  // the warps' states above are read: the stage area is free
     const size_t rbase = ((size_t)unit * sc.max_chunks + nch) * G;

@@ -120,16 +120,17 @@ __global__ void __launch_bounds__(NT, 5)
     S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * sh.sigma;
   }
 
-  // work items: the nb sealed blocks, then the residual block (item nb); the
-  // CTAs of a unit take floor or ceil((nb + 1) / gridDim.x) consecutive items
+  // work items: the nb sealed blocks, then the residual block (items nb and
+  // nb + 1 when it holds tokens); the CTAs of a unit take floor or ceil of
+  // items / gridDim.x consecutive items
   const int nch = gridDim.x;
-  const int items = sh.nb + 1;
+  const int items = sh.nb + (sh.r > 0 ? 2 : 1);  // a residual block costs about two sealed ones
   const int base = items / nch, rem = items - base * nch;
   const int i0 = chunk * base + min(chunk, rem);
   const int i1 = i0 + base + (chunk < rem ? 1 : 0);
   const int j0 = i0;
   const int nblk = max(0, min(i1, sh.nb) - i0);
-  const bool do_res = i1 > sh.nb;  // the unit's last CTA
+  const bool do_res = i0 <= sh.nb && sh.nb < i1;  // the CTA holding item nb
   if (tid == 0) {
     for (int s2 = 0; s2 < NST; ++s2) mbar_init(&S.bar[s2], 1);
     mbar_init_fence();
@@ -293,29 +294,51 @@ __global__ void __launch_bounds__(NT, 5)
   }
   if (nblk > 0) finish_ell((nblk - 1) & 1, j0 + nblk - 1);
 
-  // ---- the residual block (item nb), by the unit's last CTA: exact logits from
+  // ---- the residual block (item nb), by the CTA holding that item: exact logits from
   // the FP16 keys in device memory ----
   if (do_res) {
     float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK]
     const int r = sh.r;
     const __half* kr = t.kres + u * st.res;
     constexpr int CPL = D / 32;
-    for (int tt = warp; tt < r; tt += NW) {
-      float kf[CPL];
+    // four tokens per warp at a time: their key loads and the 4*G reductions are
+    // independent, so their latencies overlap
+    for (int t0 = 4 * warp; t0 < r; t0 += 4 * NW) {
+      float kf[4][CPL];
 #pragma unroll
-      for (int i = 0; i < CPL; i += 2) {
-        const float2 f = __half22float2(
-            *reinterpret_cast<const __half2*>(kr + (size_t)tt * D + lane * CPL + i));
-        kf[i] = f.x;
-        kf[i + 1] = f.y;
+      for (int k = 0; k < 4; ++k) {
+#pragma unroll
+        for (int i = 0; i < CPL; i += 2) {
+          float2 f = make_float2(0.f, 0.f);
+          if (t0 + k < r)
+            f = __half22float2(*reinterpret_cast<const __half2*>(kr + (size_t)(t0 + k) * D +
+                                                                 lane * CPL + i));
+          kf[k][i] = f.x;
+          kf[k][i + 1] = f.y;
+        }
       }
+      float v[4][G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = 0.f;
+      for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) v = fmaf(S.qf[h][lane * CPL + i], kf[i], v);
-        v = swarp_sum(v);
-        if (lane == 0) lg[h * BLK + tt] = v;
+        for (int h = 0; h < G; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int i = 0; i < CPL; ++i) a = fmaf(S.qf[h][lane * CPL + i], kf[k][i], a);
+          v[k][h] = a;
+        }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int h = 0; h < G; ++h) v[k][h] += __shfl_xor_sync(0xffffffffu, v[k][h], m);
+      if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            if (t0 + k < r) lg[h * BLK + t0 + k] = v[k][h];
       }
     }
     __syncthreads();
@@ -342,7 +365,8 @@ int score_chunks(const DecodeShape& sh) {
   const int units = sh.B * sh.Hkv;
   int per_unit = sh.sms * 5 / units;
   if (per_unit < 1) per_unit = 1;
-  return per_unit < sh.nb + 1 ? per_unit : sh.nb + 1;
+  const int items = sh.nb + (sh.r > 0 ? 2 : 1);
+  return per_unit < items ? per_unit : items;
 }
 
 template <int D, int G>
