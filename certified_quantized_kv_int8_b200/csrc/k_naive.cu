@@ -1,6 +1,7 @@
 // The INT8/INT4 decode path with certification off: one streaming pass over
 // Tier 1 that scores the INT8 keys, runs the online softmax and accumulates
-// the INT4 values, plus a combine that reports E_key and E_val.
+// the INT4 values; the last CTA of each (batch row, kv head) to finish merges
+// the split-K partials and reports the outputs, E_key and E_val.
 //
 // Runtime-Certified Bounded-Error Quantized Attention, Experimental Results
 // (the naive INT8/INT4 baseline, without certification) and Methodology §2
@@ -14,10 +15,10 @@
 // codes, key scales, INT4 codes, value scale/offset of one block per stage):
 // 14.5 KiB per block for head_dim 128, every byte of Tier 1 read once.
 //
-// The pass is bound by instruction issue as much as by HBM (per token and kv
-// head: 128 INT8 and 128 INT4 conversions and 2*G*head_dim multiply-adds
-// against 232 bytes), so the layout is chosen to spend few instructions
-// besides those:
+// The pass is bound by instruction issue and the FP32 pipe rather than by HBM
+// (per token and kv head: 128 INT8 and 128 INT4 conversions and 2*G*head_dim
+// multiply-adds against 232 bytes), so the layout is chosen to spend few
+// instructions besides those:
 //   * one CTA barrier per block: it publishes the block's scaled queries
 //     (double-buffered by block parity) and releases the previous block's
 //     stage to the copy engine;
@@ -32,8 +33,8 @@
 //     exponential is one exp2;
 //   * INT4 codes become floats by masking a nibble into the mantissa of 2^23
 //     (nibbles 0-4 of a word in place, 5-7 after one shift) and one packed
-//     subtraction; nibble k then carries a power-of-two factor 16^k that is
-//     divided out of its accumulator once per chunk (exact);
+//     subtraction; each nibble then carries a power-of-two factor (16^k, or
+//     16^(k-5)) that is divided out of its accumulator once per chunk (exact);
 //   * the value scale is folded into the attention weight per (token, group,
 //     head) by the softmax lanes, which also accumulate the offset term.
 #include "bulk_pipe.cuh"
@@ -122,8 +123,9 @@ __device__ __forceinline__ float nib_unscale(int k) {
 }
 
 // float offsets in the stage area where the merge of a unit's partials starts:
-// after the residual CTA's logits and statistics, after the main CTAs' per-warp
-// states (multiples of 4 floats, so the merge's float4 scratch stays aligned)
+// after the residual block's logits and statistics and after the per-warp
+// states, which a CTA may both hold there (multiples of 4 floats, so the
+// merge's float4 scratch stays aligned)
 template <int D, int G>
 struct NaiveMergeAt {
   static constexpr int RES = (G * BLK + 2 * G + 3) / 4 * 4;
@@ -155,9 +157,8 @@ __device__ double naive_e_key(double dT, double dA, double m8T) {
 
 // Arrival of one CTA of a (batch row, kv head) unit; the last of its narr
 // CTAs merges the unit's nparts partials (split-K combine; the last part is
-// the residual block's) into the outputs: the
-// outputs o / L, E_key from the largest Delta and the residual's mass, and
-// E_val = sum of eta-weighted mass / L.  Every CTA of the launch calls this
+// the residual block's) into the outputs o / L, E_key from the largest Delta
+// and the residual's mass, and E_val = sum of eta-weighted mass / L.  Every CTA of the launch calls this
 // exactly once, also after a failed wait, so the arrival counter returns to
 // zero for the next launch.
 template <int D, int G>

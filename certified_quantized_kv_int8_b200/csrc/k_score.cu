@@ -14,7 +14,7 @@
 //
 // The pass reads 136 bytes per token and kv head (128 B of codes, 8 B of
 // scales amortised) and writes 16 B of logits.  Its cost is instruction issue
-// as much as HBM, so it is laid out like the certification-off pass:
+// rather than HBM, so it is laid out like the certification-off pass:
 //   * one CTA streams consecutive blocks of one (batch row, kv head) through
 //     a ring of NST stages filled by bulk copies (codes + scales of a block);
 //   * one CTA barrier per block publishes the block's scaled queries
@@ -26,8 +26,8 @@
 //   * each warp reduces its tokens' log-sum-exp per head; the four slices
 //     merge into ell8_b after the next barrier;
 //   * logits leave through shared memory as 16-byte stores.
-// The residual block is scored exactly from its FP16 keys by one more CTA per
-// (batch row, kv head).
+// The residual block is scored exactly from its FP16 keys, after its blocks,
+// by the CTA that holds it among its work items (it counts as two).
 #include "bulk_pipe.cuh"
 #include "cqa_internal.cuh"
 
