@@ -209,23 +209,25 @@ def decision_census(cache, qs, th, w, device) -> dict:
         cache.decode(layer, qs[layer], th, outputs=o, trace=tr)
         torch.cuda.synchronize(device)
         nb = cache.length(layer) // BLOCK
+        nb_row = np.array([n // BLOCK for n in cache.row_lengths(layer)])  # ragged rows
+        own = (np.arange(nb)[None, :] < nb_row[:, None])[:, None, :]  # [B][1][nb]
         bf = tr["block_flags"].cpu().numpy()[..., :nb]  # [B][Hkv][nb]
         rg = o[3].cpu().numpy()  # [B][Hq]
         dense_h = rg.reshape(B, Hkv, G) >= 3
         unit_dense = dense_h.any(axis=2)  # [B][Hkv]
         unit_mixed = (~dense_h).any(axis=2)
-        kp = (bf & 1).astype(bool)
-        vp = (bf & 2).astype(bool)
-        c["blocks"] += int(bf.size)
-        c["blocks_per_layer"] = B * Hkv * nb
+        kp = (bf & 1).astype(bool) & own
+        vp = (bf & 2).astype(bool) & own
+        c["blocks"] += int(nb_row.sum()) * Hkv
+        c["blocks_per_layer"] = int(nb_row.sum()) * Hkv
         c["key_promoted"] += int(kp.sum())
         c["value_promoted"] += int(vp.sum())
         c["units"] += B * Hkv
         c["dense_units"] += int(unit_dense.sum())
-        c["dense_unit_blocks"] += int(unit_dense.sum()) * nb
-        c["dense_unit_nonpromoted"] += int((~kp & unit_dense[..., None]).sum())
-        c["vp_or_dense_blocks"] += int((vp | unit_dense[..., None]).sum())
-        c["int4_blocks"] += int((~vp & unit_mixed[..., None]).sum())
+        c["dense_unit_blocks"] += int((unit_dense * nb_row[:, None]).sum())
+        c["dense_unit_nonpromoted"] += int((~kp & own & unit_dense[..., None]).sum())
+        c["vp_or_dense_blocks"] += int(((vp | unit_dense[..., None]) & own).sum())
+        c["int4_blocks"] += int((~vp & own & unit_mixed[..., None]).sum())
         c["heads"] += int(rg.size)
         for r in range(5):
             c["rungs"][r] += int((rg == r).sum())
@@ -301,19 +303,31 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     wr = dataclasses.replace(w, seed=w.seed + rank)  # independent replica per rank
 
     cache = cqa.Cache(L, B, Hq, Hkv, d, max_ctx, device=device.index)
+    lens0 = sk.row_lengths(w)
     for layer in range(L):
-        K, V = sk.kv_layer(wr, layer, 0, w.ctx, device=device)
-        cache.append(layer, K, V)
+        if w.row_ctx:  # a ragged batch: each row appended on its own
+            for b, n in enumerate(lens0):
+                K, V = sk.kv_row(wr, layer, b, 0, n, device=device)
+                cache.append_row(layer, b, K, V)
+        else:
+            K, V = sk.kv_layer(wr, layer, 0, w.ctx, device=device)
+            cache.append(layer, K, V)
         del K, V
     torch.cuda.synchronize(device)
 
     # per-step inputs, resident on the device
+    def step_kv(layer, step):
+        if not w.row_ctx:
+            t = w.ctx + step
+            return sk.kv_layer(wr, layer, t, t + 1, device)
+        rows = [sk.kv_row(wr, layer, b, n + step, n + step + 1, device)
+                for b, n in enumerate(lens0)]
+        return (torch.stack([k for k, _ in rows]).contiguous(),
+                torch.stack([v for _, v in rows]).contiguous())
+
     def step_inputs(step):
         qs = [sk.queries(wr, layer, step, device) for layer in range(L)]
-        kv = []
-        if appends:
-            t = w.ctx + step
-            kv = [sk.kv_layer(wr, layer, t, t + 1, device) for layer in range(L)]
+        kv = [step_kv(layer, step) for layer in range(L)] if appends else []
         return qs, kv
 
     inputs = [step_inputs(s) for s in range(total_steps)]
@@ -469,8 +483,9 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             row["v_tol"] = v if v != float("inf") else "inf"
             row["decode_ms"] = ta.elapsed_time(tb) / 5
         vtol_sweep = rows
-    nb_total = sum(cache.length(layer) // BLOCK for layer in range(L))
-    t1_bytes = nb_total * B * Hkv * tier1_bytes_per_block(d)  # per step (lengths at the end)
+    # sealed blocks of all (layer, batch row) units per kv head, lengths at the end
+    blk_units = sum(n // BLOCK for layer in range(L) for n in cache.row_lengths(layer))
+    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d)  # per step
     peaks = measured_peaks()
     kv_gbs = t1_bytes * n_naive / n_max / 1e9 * ws
 
@@ -556,7 +571,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "peak_source": f"MEASURED_PEAKS.json hbm_gbs, of {peaks['source']}",
             "avg_launch_ms": avg, "algorithmic_bytes_per_launch": per_launch,
-            "traffic": (rec_nv["dram_bytes_per_block"] * nb_total * B * Hkv / L if rec_nv else None),
+            "traffic": (rec_nv["dram_bytes_per_block"] * blk_units * Hkv / L if rec_nv else None),
         }
         naive_roof["frac"] = naive_roof["achieved"] / naive_roof["peak"]
     res = {
@@ -575,6 +590,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         "config": {
             "workload": w.name, "layers": L, "global_batch": B * ws, "batch_per_gpu": B,
             "ctx": w.ctx, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
+            **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {}),
             "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
             "l2": "inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (
                 t1_bytes / 2 ** 30),
@@ -621,8 +637,8 @@ def oracle_sample_seconds(w: sk.Workload, layer: int, b: int, th) -> tuple[float
     """Time the CPU oracle's decode of one (layer, batch row) of the workload."""
     from oracle import Thresholds as OT
     from oracle import build_unit, decode
-    K, V = sk.kv_layer(w, layer, 0, w.ctx, device="cpu")
-    units = [build_unit(K[b, g].numpy(), V[b, g].numpy()) for g in range(w.n_kv_heads)]
+    K, V = sk.kv_row(w, layer, b, 0, sk.row_lengths(w)[b], device="cpu")
+    units = [build_unit(K[g].numpy(), V[g].numpy()) for g in range(w.n_kv_heads)]
     q = sk.queries(w, layer, 0, "cpu")[b].numpy()
     d = th.float32_rounded()
     oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
@@ -631,6 +647,13 @@ def oracle_sample_seconds(w: sk.Workload, layer: int, b: int, th) -> tuple[float
     t0 = time.perf_counter()
     decode(q, units, oth)
     return time.perf_counter() - t0, units
+
+
+def rows_per_sample(w: sk.Workload) -> float:
+    """Batch rows of a step in units of row 0 (the sampled row), by length: the
+    oracle's decode time grows with the row's length."""
+    lens = sk.row_lengths(w)
+    return sum(lens) / lens[0]
 
 
 def blas_threads() -> int:
@@ -655,16 +678,18 @@ def cpu_baseline(w: sk.Workload, th, budget_s: float = 20.0) -> dict:
         n += 1
         layer += 1
     per = statistics.mean(secs)
-    step_s = per * w.n_layers * w.batch
+    scale = w.n_layers * rows_per_sample(w)
+    step_s = per * scale
     res = {"value": 1.0 / step_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
            "sample": f"{n} of {w.n_layers * w.batch} (layer, batch row) decodes of one step, "
-                     f"{per:.2f} s each, scaled to the full step (appends not included)"}
+                     f"{per:.2f} s each, scaled to the full step (appends not included"
+                     + (", rows scaled by length)" if w.row_ctx else ")")}
     # the same oracle on one thread (one (layer, batch row) decode)
     try:
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1):
             s1, _ = oracle_sample_seconds(w, 0, 0, th)
-        res["single_thread_value"] = 1.0 / (s1 * w.n_layers * w.batch)
+        res["single_thread_value"] = 1.0 / (s1 * scale)
         res["single_thread_sample"] = f"1 (layer, batch row) decode, {s1:.2f} s, scaled"
     except ImportError:
         pass
@@ -676,10 +701,10 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
     if rank != 0:
         return None
     th = cqa_py.Thresholds(**sk.default_thresholds(w))
-    K, V = sk.kv_layer(w, 0, 0, w.ctx, device="cpu")
+    K, V = sk.kv_row(w, 0, 0, 0, sk.row_lengths(w)[0], device="cpu")
     from oracle import Thresholds as OT
     from oracle import build_unit, decode
-    units = [build_unit(K[0, g].numpy(), V[0, g].numpy()) for g in range(w.n_kv_heads)]
+    units = [build_unit(K[g].numpy(), V[g].numpy()) for g in range(w.n_kv_heads)]
     d = th.float32_rounded()
     oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
              rank_r=d["rank_r"], max_expand=d["max_expand"],
@@ -692,17 +717,20 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
         decode(qs[s], units, oth)
     el = time.perf_counter() - t0
     per = el / args.steps
-    value = 1.0 / (per * w.n_layers * w.batch)
+    scale = w.n_layers * rows_per_sample(w)
+    value = 1.0 / (per * scale)
     sample = (f"each step decodes one (layer 0, batch row 0) of the {w.n_layers}-layer, "
-              f"batch-{w.batch} step ({per:.2f} s) and is scaled by {w.n_layers * w.batch}")
+              f"batch-{w.batch} step ({per:.2f} s) and is scaled by {scale:g}"
+              + (" (rows scaled by length)" if w.row_ctx else ""))
     return {
         "metric": METRIC, "impl": "reference", "value": value, "unit": "steps/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per * w.n_layers * w.batch * 1e3, "higher_is_better": True,
+        "ms_per_step": per * scale * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "layers": w.n_layers, "global_batch": w.batch,
                    "ctx": w.ctx, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim},
+                   "head_dim": w.head_dim,
+                   **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {})},
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,

@@ -27,8 +27,8 @@ from .build import LIB
 
 __all__ = [
     "CqaError", "Thresholds", "Cache", "load_library",
-    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
-    "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
+    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_cache_row_lengths",
+    "cqa_quantize_append", "cqa_quantize_append_row", "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "PHASES", "cqa_dense_attention_noalloc",
     "cqa_set_key_prefetch", "cqa_device_status",
     "EXPORT_KCODES", "EXPORT_KSCALE", "EXPORT_VCODES", "EXPORT_VMETA", "EXPORT_ETA",
@@ -39,8 +39,8 @@ EXPORT_KCODES, EXPORT_KSCALE, EXPORT_VCODES, EXPORT_VMETA = 0, 1, 2, 3
 EXPORT_ETA, EXPORT_VRANGE, EXPORT_RESIDUAL, EXPORT_TIER2 = 4, 5, 6, 7
 
 EXPORTED_SYMBOLS = (
-    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_quantize_append",
-    "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
+    "cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length", "cqa_cache_row_lengths",
+    "cqa_quantize_append", "cqa_quantize_append_row", "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
     "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait",
 )
@@ -119,7 +119,9 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_cache_create.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(vp)]
     lib.cqa_cache_destroy.argtypes = [vp]
     lib.cqa_cache_length.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.cqa_cache_row_lengths.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32)]
     lib.cqa_quantize_append.argtypes = [vp, i32, vp, vp, i32, vp]
+    lib.cqa_quantize_append_row.argtypes = [vp, i32, i32, vp, vp, i32, vp]
     lib.cqa_decode.argtypes = [vp, i32, vp, ctypes.POINTER(_Thresholds), vp, vp, vp, vp,
                                ctypes.POINTER(_Trace), vp]
     lib.cqa_dense_reference.argtypes = [vp, i32, vp, vp, vp]
@@ -135,7 +137,8 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
-                 "cqa_quantize_append", "cqa_decode", "cqa_dense_reference",
+                 "cqa_cache_row_lengths", "cqa_quantize_append", "cqa_quantize_append_row",
+                 "cqa_decode", "cqa_dense_reference",
                  "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
                  "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait"):
         getattr(lib, name).restype = ctypes.c_int
@@ -186,11 +189,25 @@ def cqa_cache_length(handle, layer: int) -> int:
     return int(out.value)
 
 
+def cqa_cache_row_lengths(handle, layer: int, batch: int) -> list:
+    out = (ctypes.c_int32 * batch)()
+    _check(load_library().cqa_cache_row_lengths(handle, layer, out), "cqa_cache_row_lengths")
+    return [int(x) for x in out]
+
+
 def cqa_quantize_append(handle, layer, k, v, stream=None):
     """k, v: CUDA float16 [batch][n_kv_heads][n_new][head_dim]."""
     n_new = int(k.shape[2])
     return _check(load_library().cqa_quantize_append(handle, layer, _ptr(k), _ptr(v), n_new,
                                                      _stream(stream)), "cqa_quantize_append")
+
+
+def cqa_quantize_append_row(handle, layer, row, k, v, stream=None):
+    """k, v: CUDA float16 [n_kv_heads][n_new][head_dim], appended to batch row `row`."""
+    n_new = int(k.shape[1])
+    return _check(load_library().cqa_quantize_append_row(handle, layer, row, _ptr(k), _ptr(v),
+                                                         n_new, _stream(stream)),
+                  "cqa_quantize_append_row")
 
 
 def cqa_decode(handle, layer, q, th: Thresholds, out, e_key, e_val, rung, trace=None, stream=None):
@@ -307,13 +324,23 @@ class Cache:
         return cqa_profile_end(self.handle)
 
     def length(self, layer):
+        """Tokens of the layer's longest batch row."""
         return cqa_cache_length(self.handle, layer)
+
+    def row_lengths(self, layer):
+        return cqa_cache_row_lengths(self.handle, layer, self.batch)
 
     def append(self, layer, k, v, stream=None):
         B, H, d = self.batch, self.n_kv_heads, self.head_dim
         _dev(k, torch.float16, (B, H, k.shape[2], d), "k")
         _dev(v, torch.float16, (B, H, k.shape[2], d), "v")
         return cqa_quantize_append(self.handle, layer, k, v, stream)
+
+    def append_row(self, layer, row, k, v, stream=None):
+        H, d = self.n_kv_heads, self.head_dim
+        _dev(k, torch.float16, (H, k.shape[1], d), "k")
+        _dev(v, torch.float16, (H, k.shape[1], d), "v")
+        return cqa_quantize_append_row(self.handle, layer, row, k, v, stream)
 
     def alloc_outputs(self):
         dev = torch.device("cuda", self.device)
@@ -353,21 +380,34 @@ class Cache:
         return out
 
     def export(self, layer, what):
-        """Tier-1 array of `layer` as a numpy array shaped per include/cqa.h."""
-        B, H, d = self.batch, self.n_kv_heads, self.head_dim
-        T = self.length(layer)
-        nb, r = T // 64, T % 64
-        spec = {
-            EXPORT_KCODES: (np.int8, (B, H, nb, 64, d)),
-            EXPORT_KSCALE: (np.float32, (B, H, nb, d)),
-            EXPORT_VCODES: (np.uint8, (B, H, nb, 64, d // 2)),
-            EXPORT_VMETA: (np.float32, (B, H, nb, 64, d // 32, 2)),
-            EXPORT_ETA: (np.float32, (B, H, nb)),
-            EXPORT_VRANGE: (np.float32, (B, H, 2, d)),
-            EXPORT_RESIDUAL: (np.float16, (B, H, 2, r, d)),
-            EXPORT_TIER2: (np.float16, (B, H, 2, T, d)),
-        }[what]
-        dst = np.empty(spec[1], dtype=spec[0])
-        n = cqa_debug_export(self.handle, layer, what, dst)
-        assert n == dst.nbytes
-        return dst
+        """Tier-1 array of `layer` as a numpy array shaped per include/cqa.h; when the
+        rows' extents differ (a ragged layer), a list of per-row arrays (each
+        without the batch axis)."""
+        H, d = self.n_kv_heads, self.head_dim
+        lens = self.row_lengths(layer)
+
+        def spec(T):
+            nb, r = T // 64, T % 64
+            return {
+                EXPORT_KCODES: (np.int8, (H, nb, 64, d)),
+                EXPORT_KSCALE: (np.float32, (H, nb, d)),
+                EXPORT_VCODES: (np.uint8, (H, nb, 64, d // 2)),
+                EXPORT_VMETA: (np.float32, (H, nb, 64, d // 32, 2)),
+                EXPORT_ETA: (np.float32, (H, nb)),
+                EXPORT_VRANGE: (np.float32, (H, 2, d)),
+                EXPORT_RESIDUAL: (np.float16, (H, 2, r, d)),
+                EXPORT_TIER2: (np.float16, (H, 2, T, d)),
+            }[what]
+
+        specs = [spec(T) for T in lens]
+        sizes = [int(np.prod(sh)) * np.dtype(dt).itemsize for dt, sh in specs]
+        flat = np.empty(sum(sizes), dtype=np.uint8)
+        n = cqa_debug_export(self.handle, layer, what, flat)
+        assert n == flat.nbytes
+        rows, off = [], 0
+        for (dt, sh), size in zip(specs, sizes):
+            rows.append(flat[off:off + size].view(dt).reshape(sh))
+            off += size
+        if len({sh for _, sh in specs}) == 1:  # equal shapes: one array
+            return np.stack(rows)
+        return rows

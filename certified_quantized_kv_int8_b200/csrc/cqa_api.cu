@@ -42,7 +42,9 @@ struct cqa_cache {
   Strides st;
   Tier1 t;
   Scratch sc;
-  int32_t* len;  // host: tokens per layer
+  int32_t* len;        // host [n_layers][batch]: tokens of each batch row
+  int32_t* lens_dev;   // device copy of len, written by the append kernels in stream order
+  uint32_t* seal_gen;  // host [n_layers]: count of appends that sealed a block in the layer
   void* k2_host;
   void* v2_host;
   size_t tier2_bytes;  // per tier-2 array
@@ -60,7 +62,8 @@ struct cqa_cache {
   cudaStream_t side;   // copy stream
   __half* kstage[2];   // [B*Hkv][max_ctx][d] device copies of one layer's Tier-2 keys
   int stage_layer[2];  // layer held by each slot, -1 none
-  int stage_nb[2];     // sealed blocks copied into the slot
+  int stage_nb[2];     // sealed blocks copied into the slot (of the layer's longest row)
+  uint32_t stage_gen[2];  // seal_gen of the layer when the slot was filled
   cudaEvent_t ev_ready[2], ev_free[2], ev_main;
   int32_t* promo_host; // [n_layers * B * Hkv] promoted blocks of the last decode (mapped)
   int32_t* promo_dev;
@@ -98,19 +101,45 @@ void chunking(int units, int nb, int sms, int* chunk_blocks, int* nchunks) {
 
 int max_chunks_for(int units, int sms) { return (target_ctas(sms) + units - 1) / units + 1; }
 
-DecodeShape shape_of(const cqa_cache* c, int T) {
+const int32_t* row_lens(const cqa_cache* c, int layer) {
+  return c->len + (size_t)layer * c->cfg.batch;
+}
+
+int max_len(const cqa_cache* c, int layer) {
+  const int32_t* L = row_lens(c, layer);
+  int m = 0;
+  for (int b = 0; b < c->cfg.batch; ++b) m = L[b] > m ? L[b] : m;
+  return m;
+}
+
+int min_len(const cqa_cache* c, int layer) {
+  const int32_t* L = row_lens(c, layer);
+  int m = L[0];
+  for (int b = 1; b < c->cfg.batch; ++b) m = L[b] < m ? L[b] : m;
+  return m;
+}
+
+// Grids cover the longest row; each CTA reads its own row's length on the device.
+DecodeShape shape_of(const cqa_cache* c, int layer) {
   DecodeShape sh;
   sh.B = c->cfg.batch;
   sh.Hq = c->cfg.n_q_heads;
   sh.Hkv = c->cfg.n_kv_heads;
   sh.G = c->G;
   sh.d = c->cfg.head_dim;
-  sh.nb = T / BLK;
-  sh.r = T - sh.nb * BLK;
+  sh.nb_max = 0;
+  sh.items_max = 1;
+  const int32_t* L = row_lens(c, layer);
+  for (int b = 0; b < sh.B; ++b) {
+    const int nb = L[b] / BLK, r = L[b] - (L[b] / BLK) * BLK;
+    if (nb > sh.nb_max) sh.nb_max = nb;
+    if (row_items(nb, r) > sh.items_max) sh.items_max = row_items(nb, r);
+  }
   sh.nbm = c->nbm;
+  sh.lens = c->lens_dev + (size_t)layer * sh.B;
   sh.sigma = (float)(1.0 / sqrt((double)sh.d));
   sh.sms = c->sms;
-  chunking(sh.B * sh.Hkv, sh.nb, sh.sms, &sh.chunk_blocks, &sh.nchunks);
+  chunking(sh.B * sh.Hkv, sh.nb_max, sh.sms, &sh.chunk_blocks, &sh.nchunks);
   return sh;
 }
 
@@ -161,51 +190,72 @@ cudaError_t run_phase(cqa_cache* c, int phase, cudaStream_t s, int nlaunch, F&& 
 }
 
 // Fraction of the layer's sealed blocks its last decode promoted (-1 unknown).
-double last_promoted_fraction(const cqa_cache* c, int layer, int nb) {
-  const size_t units = (size_t)c->cfg.batch * c->cfg.n_kv_heads;
+double last_promoted_fraction(const cqa_cache* c, int layer) {
+  const int Hkv = c->cfg.n_kv_heads;
+  const size_t units = (size_t)c->cfg.batch * Hkv;
   const volatile int32_t* p = c->promo_host + (size_t)layer * units;
-  long long n = 0;
+  const int32_t* L = row_lens(c, layer);
+  long long n = 0, total = 0;
   for (size_t i = 0; i < units; ++i) {
     const int32_t v = p[i];
     if (v < 0) return -1.0;
     n += v;
+    total += L[i / Hkv] / BLK;
   }
-  return nb > 0 ? (double)n / ((double)units * nb) : -1.0;
+  return total > 0 ? (double)n / (double)total : -1.0;
 }
 
 bool want_prefetch(const cqa_cache* c, int layer) {
   if (c->pref_mode == 0) return false;
-  const int nb = c->len[layer] / BLK;
-  if (nb == 0) return false;
+  if (max_len(c, layer) / BLK == 0) return false;
   if (c->pref_mode == 2) return true;
-  return last_promoted_fraction(c, layer, nb) >= c->pref_min_frac;
+  return last_promoted_fraction(c, layer) >= c->pref_min_frac;
 }
 
+// The slot holding `layer`'s keys as they are now (no block sealed since), or -1.
 int staged_slot(const cqa_cache* c, int layer) {
   for (int i = 0; i < 2; ++i)
-    if (c->stage_layer[i] == layer) return i;
+    if (c->stage_layer[i] == layer && c->stage_gen[i] == c->seal_gen[layer]) return i;
   return -1;
 }
 
 // Copy the sealed blocks of `layer`'s Tier-2 keys into a device slot on the
 // copy stream, after all work already queued on `s` (the appends that wrote
-// them) and after the slot's last reader.  Returns the slot or -1.
+// them) and after the slot's last reader.  Each batch row copies its own
+// sealed blocks (one copy for all rows when their block counts agree).
+// Returns the slot or -1.
 int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
-  const int nb = c->len[layer] / BLK;
+  const int nb = max_len(c, layer) / BLK;
   if (nb == 0) return -1;
   int slot = staged_slot(c, layer);
-  if (slot >= 0 && c->stage_nb[slot] == nb) return slot;
-  if (slot < 0) slot = (avoid_slot == 0) ? 1 : 0;
-  const size_t units = (size_t)c->cfg.batch * c->cfg.n_kv_heads;
+  if (slot >= 0) return slot;
+  slot = (avoid_slot == 0) ? 1 : 0;
+  const int B = c->cfg.batch, Hkv = c->cfg.n_kv_heads;
+  const size_t units = (size_t)B * Hkv;
   const size_t pitch = c->st.tier2 * 2;
+  const size_t blk_bytes = (size_t)BLK * c->cfg.head_dim * 2;
   const char* src = (const char*)c->k2_host + (size_t)layer * units * pitch;
+  const int32_t* L = row_lens(c, layer);
+  bool same = true;
+  for (int b = 1; b < B; ++b) same = same && (L[b] / BLK == L[0] / BLK);
   if (cudaEventRecord(c->ev_main, s) != cudaSuccess) return -1;
   if (cudaStreamWaitEvent(c->side, c->ev_main, 0) != cudaSuccess) return -1;
   if (cudaStreamWaitEvent(c->side, c->ev_free[slot], 0) != cudaSuccess) return -1;
   const int timed = c->prof_on ? 1 : 0;
   cudaError_t e = run_phase(c, CQA_PHASE_PREFETCH, c->side, timed, [&] {
-    return cudaMemcpy2DAsync(c->kstage[slot], pitch, src, pitch, (size_t)nb * BLK * c->cfg.head_dim * 2,
-                             units, cudaMemcpyHostToDevice, c->side);
+    if (same)
+      return cudaMemcpy2DAsync(c->kstage[slot], pitch, src, pitch, (size_t)nb * blk_bytes, units,
+                               cudaMemcpyHostToDevice, c->side);
+    for (int b = 0; b < B; ++b) {
+      const int nbr = L[b] / BLK;
+      if (nbr == 0) continue;
+      const size_t off = (size_t)b * Hkv * pitch;
+      const cudaError_t e2 =
+          cudaMemcpy2DAsync((char*)c->kstage[slot] + off, pitch, src + off, pitch,
+                            (size_t)nbr * blk_bytes, Hkv, cudaMemcpyHostToDevice, c->side);
+      if (e2 != cudaSuccess) return e2;
+    }
+    return cudaSuccess;
   });
   if (e != cudaSuccess || cudaEventRecord(c->ev_ready[slot], c->side) != cudaSuccess) {
     c->stage_layer[slot] = -1;
@@ -213,6 +263,7 @@ int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
   }
   c->stage_layer[slot] = layer;
   c->stage_nb[slot] = nb;
+  c->stage_gen[slot] = c->seal_gen[layer];
   return slot;
 }
 
@@ -309,6 +360,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   const size_t o_px = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
   const size_t o_cnt = take((size_t)c.batch * c.n_kv_heads * sizeof(int));
   const size_t o_dcnt = take((size_t)c.batch * 2 * sizeof(int));
+  const size_t o_lens = take((size_t)c.n_layers * c.batch * sizeof(int32_t));
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     cudaGetLastError();
@@ -341,6 +393,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->sc.part_x = (float*)(bp + o_px);
   cc->sc.cnt = (int*)(bp + o_cnt);
   cc->sc.dcnt = (int*)(bp + o_dcnt);
+  cc->lens_dev = (int32_t*)(bp + o_lens);
   cc->sc.ls = ls;
   cc->sc.max_chunks = (int)max_chunks;
 
@@ -373,8 +426,9 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->t.k2 = (__half*)kd;
   cc->t.v2 = (__half*)vd;
 
-  cc->len = (int32_t*)calloc((size_t)c.n_layers, sizeof(int32_t));
-  if (!cc->len) {
+  cc->len = (int32_t*)calloc((size_t)c.n_layers * c.batch, sizeof(int32_t));
+  cc->seal_gen = (uint32_t*)calloc((size_t)c.n_layers, sizeof(uint32_t));
+  if (!cc->len || !cc->seal_gen) {
     cqa_cache_destroy(cc);
     return CQA_ERR_OOM;
   }
@@ -442,13 +496,46 @@ int cqa_cache_destroy(cqa_cache* cc) {
   delete cc->prof_events;
   delete cc->prof_phase;
   free(cc->len);
+  free(cc->seal_gen);
   delete cc;
   return rc;
 }
 
 int cqa_cache_length(const cqa_cache* cc, int layer, int32_t* out_len) {
   if (!cc || !out_len || layer < 0 || layer >= cc->cfg.n_layers) return CQA_ERR_INVALID_ARG;
-  *out_len = cc->len[layer];
+  *out_len = max_len(cc, layer);
+  return CQA_OK;
+}
+
+int cqa_cache_row_lengths(const cqa_cache* cc, int layer, int32_t* out_lens) {
+  if (!cc || !out_lens || layer < 0 || layer >= cc->cfg.n_layers) return CQA_ERR_INVALID_ARG;
+  memcpy(out_lens, row_lens(cc, layer), (size_t)cc->cfg.batch * sizeof(int32_t));
+  return CQA_OK;
+}
+
+// Append n_new tokens to `nrows` consecutive batch rows from `row0` that all
+// hold T_old tokens; k, v: [nrows][n_kv_heads][n_new][head_dim].
+static int append_rows(cqa_cache* cc, int layer, int row0, int nrows, const __half* kh,
+                       const __half* vh, int n_new, cudaStream_t s) {
+  const int B = cc->cfg.batch, Hkv = cc->cfg.n_kv_heads, d = cc->cfg.head_dim;
+  int32_t* L = cc->len + (size_t)layer * B;
+  const int T_old = L[row0];
+  const int T_new = T_old + n_new;
+  const int unit0 = (layer * B + row0) * Hkv;
+  const int nb_old = T_old / BLK, nb_new = T_new / BLK;
+  int32_t* lens_rows = cc->lens_dev + (size_t)layer * B + row0;
+  cudaError_t e = run_phase(cc, CQA_PHASE_APPEND_SEAL, s, nb_new > nb_old ? 1 : 0, [&] {
+    return launch_seal(cc->t, cc->st, unit0, nrows, Hkv, d, kh, vh, T_old, n_new, nb_old, nb_new,
+                       s);
+  });
+  if (e == cudaSuccess)
+    e = run_phase(cc, CQA_PHASE_APPEND_TAIL, s, 1, [&] {
+      return launch_append_tail(cc->t, cc->st, unit0, nrows, Hkv, d, kh, vh, T_old, n_new, nb_new,
+                                lens_rows, s);
+    });
+  if (e != cudaSuccess) return CQA_ERR_CUDA;
+  for (int b = row0; b < row0 + nrows; ++b) L[b] = T_new;
+  if (nb_new > nb_old) ++cc->seal_gen[layer];
   return CQA_OK;
 }
 
@@ -457,27 +544,40 @@ int cqa_quantize_append(cqa_cache* cc, int layer, const void* k, const void* v, 
   if (!cc || layer < 0 || layer >= cc->cfg.n_layers || n_new < 0) return CQA_ERR_INVALID_ARG;
   if (n_new == 0) return CQA_OK;
   if (!k || !v || !aligned16(k) || !aligned16(v)) return CQA_ERR_INVALID_ARG;
-  const int T_old = cc->len[layer];
-  if ((long long)T_old + n_new > cc->cfg.max_ctx) return CQA_ERR_CAPACITY;
-  const int T_new = T_old + n_new;
+  if ((long long)max_len(cc, layer) + n_new > cc->cfg.max_ctx) return CQA_ERR_CAPACITY;
   DeviceGuard dg(cc->cfg.device);
   if (!dg.ok) return CQA_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  const int B = cc->cfg.batch, Hkv = cc->cfg.n_kv_heads, d = cc->cfg.head_dim;
-  const int unit0 = layer * B * Hkv;
-  const int nb_old = T_old / BLK, nb_new = T_new / BLK;
+  const int B = cc->cfg.batch;
+  const size_t row_elems = (size_t)cc->cfg.n_kv_heads * n_new * cc->cfg.head_dim;
   const __half* kh = (const __half*)k;
   const __half* vh = (const __half*)v;
-  cudaError_t e = run_phase(cc, CQA_PHASE_APPEND_SEAL, s, nb_new > nb_old ? 1 : 0, [&] {
-    return launch_seal(cc->t, cc->st, unit0, B, Hkv, d, kh, vh, T_old, n_new, nb_old, nb_new, s);
-  });
-  if (e == cudaSuccess)
-    e = run_phase(cc, CQA_PHASE_APPEND_TAIL, s, 1, [&] {
-      return launch_append_tail(cc->t, cc->st, unit0, B, Hkv, d, kh, vh, T_old, n_new, nb_new, s);
-    });
-  if (e != cudaSuccess) return CQA_ERR_CUDA;
-  cc->len[layer] = T_new;
+  // runs of consecutive rows of equal length share one launch (all rows, when
+  // the batch is not ragged)
+  const int32_t* L = row_lens(cc, layer);
+  for (int b0 = 0; b0 < B;) {
+    int b1 = b0 + 1;
+    while (b1 < B && L[b1] == L[b0]) ++b1;
+    const int rc = append_rows(cc, layer, b0, b1 - b0, kh + b0 * row_elems, vh + b0 * row_elems,
+                               n_new, s);
+    if (rc != CQA_OK) return rc;
+    b0 = b1;
+  }
   return CQA_OK;
+}
+
+int cqa_quantize_append_row(cqa_cache* cc, int layer, int row, const void* k, const void* v,
+                            int n_new, void* stream) {
+  if (!cc || layer < 0 || layer >= cc->cfg.n_layers || row < 0 || row >= cc->cfg.batch ||
+      n_new < 0)
+    return CQA_ERR_INVALID_ARG;
+  if (n_new == 0) return CQA_OK;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return CQA_ERR_INVALID_ARG;
+  if ((long long)row_lens(cc, layer)[row] + n_new > cc->cfg.max_ctx) return CQA_ERR_CAPACITY;
+  DeviceGuard dg(cc->cfg.device);
+  if (!dg.ok) return CQA_ERR_CUDA;
+  return append_rows(cc, layer, row, 1, (const __half*)k, (const __half*)v, n_new,
+                     (cudaStream_t)stream);
 }
 
 static int copy_trace(cqa_cache* cc, const DecodeShape& sh, const cqa_trace* tr, cudaStream_t s) {
@@ -492,10 +592,10 @@ static int copy_trace(cqa_cache* cc, const DecodeShape& sh, const cqa_trace* tr,
   cp2(tr->kstar, cc->sc.kstar, 4, rows, rows, 1);
   cp2(tr->head_flags, cc->sc.hflags, 1, rows, rows, 1);
   cp2(tr->ell_res, cc->sc.ell_res, 4, rows, rows, 1);
-  cp2(tr->block_flags, cc->sc.bflags, 1, sh.nb, sh.nbm, (size_t)sh.B * sh.Hkv);
-  cp2(tr->ell8, cc->sc.ell8, 4, sh.nb, sh.nbm, rows);
-  cp2(tr->ell16, cc->sc.ell16, 4, sh.nb, sh.nbm, rows);
-  cp2(tr->delta, cc->sc.delta, 4, sh.nb, sh.nbm, rows);
+  cp2(tr->block_flags, cc->sc.bflags, 1, sh.nb_max, sh.nbm, (size_t)sh.B * sh.Hkv);
+  cp2(tr->ell8, cc->sc.ell8, 4, sh.nb_max, sh.nbm, rows);
+  cp2(tr->ell16, cc->sc.ell16, 4, sh.nb_max, sh.nbm, rows);
+  cp2(tr->delta, cc->sc.delta, 4, sh.nb_max, sh.nbm, rows);
   return e == cudaSuccess ? CQA_OK : CQA_ERR_CUDA;
 }
 
@@ -509,12 +609,11 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   if (!(tv.tau_cov >= 0.f) || tv.max_expand < 0 || tv.rank_r < 0 || isnan(tv.eps_key) ||
       isnan(tv.v_tol) || isnan(tv.eps_val) || isnan(tv.layer_dense_frac))
     return CQA_ERR_INVALID_ARG;
-  const int T = cc->len[layer];
-  if (T == 0) return CQA_ERR_EMPTY;
+  if (min_len(cc, layer) == 0) return CQA_ERR_EMPTY;
   DeviceGuard dg(cc->cfg.device);
   if (!dg.ok) return CQA_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  const DecodeShape sh = shape_of(cc, T);
+  const DecodeShape sh = shape_of(cc, layer);
   if (sh.nchunks > cc->sc.max_chunks) return CQA_ERR_INVALID_ARG;
   const int unit0 = layer * sh.B * sh.Hkv;
   double need = ceil((double)tv.layer_dense_frac * sh.Hq);
@@ -527,7 +626,6 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   int slot = -1;
   if (!naive) {
     slot = staged_slot(cc, layer);
-    if (slot >= 0 && cc->stage_nb[slot] != sh.nb) slot = -1;
     if (slot < 0 && want_prefetch(cc, layer)) slot = issue_prefetch(cc, layer, -1, s);
     // the next layer's keys, copied while this layer runs: the copy shares the
     // host link with this layer's value pass, which keeps the link busy through
@@ -553,14 +651,14 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
     e = run_phase(cc, CQA_PHASE_SELECT, s, 1,
                   [&] { return launch_select(cc->t, cc->st, unit0, sh, tv, cc->sc, s); });
   if (e == cudaSuccess && slot >= 0) e = cudaStreamWaitEvent(s, cc->ev_ready[slot], 0);
-  if (e == cudaSuccess && !naive && sh.nb > 0)
+  if (e == cudaSuccess && !naive && sh.nb_max > 0)
     e = run_phase(cc, CQA_PHASE_PROMOTE, s, 1, [&] {
       return launch_promote(cc->t, cc->st, unit0, sh, qh, cc->sc, 0, kstage, stage_nb, s);
     });
   if (e == cudaSuccess)
     e = run_phase(cc, CQA_PHASE_DECIDE, s, 1,
                   [&] { return launch_decide(sh, tv, need_dense, cc->sc, s); });
-  if (e == cudaSuccess && !naive && sh.nb > 0)
+  if (e == cudaSuccess && !naive && sh.nb_max > 0)
     e = run_phase(cc, CQA_PHASE_DENSE_KEYS, s, 1, [&] {
       return launch_promote(cc->t, cc->st, unit0, sh, qh, cc->sc, 1, kstage, stage_nb, s);
     });
@@ -588,12 +686,11 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
 int cqa_dense_reference(cqa_cache* cc, int layer, const void* q, float* out, void* stream) {
   if (!cc || layer < 0 || layer >= cc->cfg.n_layers || !q || !out) return CQA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return CQA_ERR_INVALID_ARG;
-  const int T = cc->len[layer];
-  if (T == 0) return CQA_ERR_EMPTY;
+  if (min_len(cc, layer) == 0) return CQA_ERR_EMPTY;
   DeviceGuard dg(cc->cfg.device);
   if (!dg.ok) return CQA_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  const DecodeShape sh = shape_of(cc, T);
+  const DecodeShape sh = shape_of(cc, layer);
   const int unit0 = layer * sh.B * sh.Hkv;
   cudaError_t e = run_phase(cc, CQA_PHASE_DENSE_ATTEND, s, 1, [&] {
     return launch_attend(cc->t, cc->st, unit0, sh, (const __half*)q, cc->sc, 2, s);
@@ -608,47 +705,62 @@ int cqa_dense_reference(cqa_cache* cc, int layer, const void* q, float* out, voi
 int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t bytes) {
   if (!cc || layer < 0 || layer >= cc->cfg.n_layers) return CQA_ERR_INVALID_ARG;
   const int B = cc->cfg.batch, Hkv = cc->cfg.n_kv_heads, d = cc->cfg.head_dim;
-  const int T = cc->len[layer];
-  const int nb = T / BLK, r = T - nb * BLK;
+  const int32_t* L = row_lens(cc, layer);
   const size_t units = (size_t)B * Hkv;
   const size_t unit0 = (size_t)layer * units;
   const Strides& st = cc->st;
   const char* srcs[2] = {nullptr, nullptr};
-  size_t per_unit = 0, stride = 0;  // bytes
+  size_t stride = 0;  // bytes between units
   bool host_src = false;
   int parts = 1;
   switch (what) {
-    case CQA_EXPORT_KCODES: srcs[0] = (const char*)cc->t.kcodes; per_unit = (size_t)nb * BLK * d; stride = st.kcodes; break;
-    case CQA_EXPORT_KSCALE: srcs[0] = (const char*)cc->t.kscale; per_unit = (size_t)nb * d * 4; stride = st.kscale * 4; break;
-    case CQA_EXPORT_VCODES: srcs[0] = (const char*)cc->t.vcodes; per_unit = (size_t)nb * BLK * d / 2; stride = st.vcodes; break;
-    case CQA_EXPORT_VMETA: srcs[0] = (const char*)cc->t.vmeta; per_unit = (size_t)nb * BLK * (d / VG) * 8; stride = st.vmeta * 4; break;
-    case CQA_EXPORT_ETA: srcs[0] = (const char*)cc->t.eta; per_unit = (size_t)nb * 4; stride = st.eta * 4; break;
-    case CQA_EXPORT_VRANGE: srcs[0] = (const char*)cc->t.vrange; per_unit = (size_t)2 * d * 4; stride = st.vrange * 4; break;
+    case CQA_EXPORT_KCODES: srcs[0] = (const char*)cc->t.kcodes; stride = st.kcodes; break;
+    case CQA_EXPORT_KSCALE: srcs[0] = (const char*)cc->t.kscale; stride = st.kscale * 4; break;
+    case CQA_EXPORT_VCODES: srcs[0] = (const char*)cc->t.vcodes; stride = st.vcodes; break;
+    case CQA_EXPORT_VMETA: srcs[0] = (const char*)cc->t.vmeta; stride = st.vmeta * 4; break;
+    case CQA_EXPORT_ETA: srcs[0] = (const char*)cc->t.eta; stride = st.eta * 4; break;
+    case CQA_EXPORT_VRANGE: srcs[0] = (const char*)cc->t.vrange; stride = st.vrange * 4; break;
     case CQA_EXPORT_RESIDUAL:
       srcs[0] = (const char*)cc->t.kres; srcs[1] = (const char*)cc->t.vres;
-      per_unit = (size_t)r * d * 2; stride = st.res * 2; parts = 2;
+      stride = st.res * 2; parts = 2;
       break;
     case CQA_EXPORT_TIER2:
       srcs[0] = (const char*)cc->k2_host; srcs[1] = (const char*)cc->v2_host;
-      per_unit = (size_t)T * d * 2; stride = st.tier2 * 2; parts = 2;
+      stride = st.tier2 * 2; parts = 2;
       host_src = true;
       break;
     default: return CQA_ERR_INVALID_ARG;
   }
-  const size_t total = units * parts * per_unit;
+  // bytes of one unit's part: each batch row exports its own extent
+  auto part_bytes = [&](int T) -> size_t {
+    const size_t nb = (size_t)(T / BLK), r = (size_t)(T - (T / BLK) * BLK);
+    switch (what) {
+      case CQA_EXPORT_KCODES: return nb * BLK * d;
+      case CQA_EXPORT_KSCALE: return nb * d * 4;
+      case CQA_EXPORT_VCODES: return nb * BLK * d / 2;
+      case CQA_EXPORT_VMETA: return nb * BLK * (d / VG) * 8;
+      case CQA_EXPORT_ETA: return nb * 4;
+      case CQA_EXPORT_VRANGE: return (size_t)2 * d * 4;
+      case CQA_EXPORT_RESIDUAL: return r * d * 2;
+      default: return (size_t)T * d * 2;  // CQA_EXPORT_TIER2
+    }
+  };
+  size_t total = 0;
+  for (int b = 0; b < B; ++b) total += (size_t)Hkv * parts * part_bytes(L[b]);
   if (!dst && bytes == 0) return (int64_t)total;
   if (!dst || bytes != total) return CQA_ERR_INVALID_ARG;
   DeviceGuard dg(cc->cfg.device);
   if (!dg.ok || cudaDeviceSynchronize() != cudaSuccess) return CQA_ERR_CUDA;
-  char* out = (char*)dst;
+  char* dp = (char*)dst;
   for (size_t uu = 0; uu < units; ++uu) {
-    for (int p = 0; p < parts; ++p) {
+    const int T = L[uu / Hkv];
+    const size_t per_unit = part_bytes(T);
+    for (int p = 0; p < parts; ++p, dp += per_unit) {
       const char* sp = srcs[p] + (unit0 + uu) * stride;
-      char* dp = out + (uu * parts + p) * per_unit;
       if (per_unit == 0) continue;
       if (host_src) {
         // sealed tokens from Tier 2; the residual block's from device memory
-        const size_t sealed = (size_t)nb * BLK * d * 2;
+        const size_t sealed = (size_t)(T / BLK) * BLK * d * 2;
         memcpy(dp, sp, sealed);
         const char* rs = (const char*)(p == 0 ? cc->t.kres : cc->t.vres) + (unit0 + uu) * st.res * 2;
         if (per_unit > sealed &&

@@ -91,11 +91,27 @@ struct Scratch {
   int max_chunks;
 };
 
+// Shape of one decode call.  Batch rows may hold different lengths: grids are
+// sized for the longest row (nb_max sealed blocks) and every CTA reads the
+// length of its own row from `lens`.
 struct DecodeShape {
-  int B, Hq, Hkv, G, d, nb, r, nbm, nchunks, chunk_blocks;
-  int sms;  // streaming multiprocessors of the cache's device (grid sizing)
+  int B, Hq, Hkv, G, d, nb_max, nbm, nchunks, chunk_blocks;
+  int items_max;        // max over rows of the streaming passes' work items (see row_items)
+  int sms;              // streaming multiprocessors of the cache's device (grid sizing)
+  const int32_t* lens;  // device [B]: tokens held by each batch row of the layer
   float sigma;
 };
+
+// Sealed blocks and residual tokens of batch row b.
+__device__ __forceinline__ void row_blocks(const DecodeShape& sh, int b, int& nb, int& r) {
+  const int T = __ldg(sh.lens + b);
+  nb = T / BLK;
+  r = T - nb * BLK;
+}
+
+// Work items of a row in the streaming passes: its sealed blocks, then the
+// residual block, which costs about two sealed ones when it holds tokens.
+__host__ __device__ __forceinline__ int row_items(int nb, int r) { return nb + (r > 0 ? 2 : 1); }
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
 // again only when a launch needs more than already granted: the attribute
@@ -106,9 +122,10 @@ cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
 cudaError_t launch_seal(const Tier1& t, const Strides& st, int layer_unit0, int B, int Hkv, int d,
                         const __half* knew, const __half* vnew, int T_old, int n_new, int nb_old,
                         int nb_new, cudaStream_t s);
+// also stores T_old + n_new as the length of each of the B rows (lens_rows[0..B))
 cudaError_t launch_append_tail(const Tier1& t, const Strides& st, int layer_unit0, int B, int Hkv,
                                int d, const __half* knew, const __half* vnew, int T_old,
-                               int n_new, int nb_new, cudaStream_t s);
+                               int n_new, int nb_new, int32_t* lens_rows, cudaStream_t s);
 cudaError_t launch_score(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
                          const __half* q, const Scratch& sc, cudaStream_t s);
 // mode 0: promoted blocks (exact logits in place, ell16); 1: the other blocks

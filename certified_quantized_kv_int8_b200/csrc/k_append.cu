@@ -145,15 +145,18 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
 }
 
 // grid (ceil(n_new/64), B*Hkv), 256 threads: residual slots, per-channel
-// value range.
+// value range, and the rows' new length (read by the decode kernels).
 template <int D>
 __global__ void __launch_bounds__(256) append_tail_kernel(Tier1 t, Strides st, int unit0,
                                                           const __half* __restrict__ knew,
                                                           const __half* __restrict__ vnew,
-                                                          int T_old, int n_new, int nb_new) {
+                                                          int T_old, int n_new, int nb_new,
+                                                          int32_t* __restrict__ lens_rows,
+                                                          int Hkv) {
   constexpr int C8 = D / 8;
   const int ug = blockIdx.y;
   const size_t u = (size_t)unit0 + ug;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && ug % Hkv == 0) lens_rows[ug / Hkv] = T_old + n_new;
   const int i0 = blockIdx.x * BLK;
   const int n = min(BLK, n_new - i0);
   for (int e = threadIdx.x; e < n * C8; e += blockDim.x) {
@@ -197,12 +200,14 @@ cudaError_t launch_seal(const Tier1& t, const Strides& st, int unit0, int B, int
 
 cudaError_t launch_append_tail(const Tier1& t, const Strides& st, int unit0, int B, int Hkv,
                                int d, const __half* knew, const __half* vnew, int T_old,
-                               int n_new, int nb_new, cudaStream_t s) {
+                               int n_new, int nb_new, int32_t* lens_rows, cudaStream_t s) {
   dim3 grid((n_new + BLK - 1) / BLK, B * Hkv);
   if (d == 128)
-    append_tail_kernel<128><<<grid, 256, 0, s>>>(t, st, unit0, knew, vnew, T_old, n_new, nb_new);
+    append_tail_kernel<128><<<grid, 256, 0, s>>>(t, st, unit0, knew, vnew, T_old, n_new, nb_new,
+                                                 lens_rows, Hkv);
   else
-    append_tail_kernel<64><<<grid, 256, 0, s>>>(t, st, unit0, knew, vnew, T_old, n_new, nb_new);
+    append_tail_kernel<64><<<grid, 256, 0, s>>>(t, st, unit0, knew, vnew, T_old, n_new, nb_new,
+                                                lens_rows, Hkv);
   return cudaGetLastError();
 }
 

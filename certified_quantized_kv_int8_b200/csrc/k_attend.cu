@@ -95,8 +95,10 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
   const size_t u = (size_t)unit0 + unit;
   const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
   const int chunk = blockIdx.x;
+  int nb, rr;
+  row_blocks(sh, b, nb, rr);
   const int j0 = chunk * sh.chunk_blocks;
-  const int j1 = min(sh.nb, j0 + sh.chunk_blocks);
+  const int j1 = min(nb, j0 + sh.chunk_blocks);  // j0 >= j1 past the end of a shorter row
 
   // per head: exact (dense) or certified mixed attention
   bool dh[G];
@@ -144,13 +146,13 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
   }
 
   const uint8_t* bf = sc.bflags + ((size_t)b * sh.Hkv + g) * sh.nbm;
-  const int jstart = (chunk == 0 && sh.r > 0) ? -1 : j0;  // -1 = the residual block
+  const int jstart = (chunk == 0 && rr > 0) ? -1 : j0;  // -1 = the residual block
   for (int j = jstart; j < j1; ++j) {
     const bool resid = j < 0;
     const uint8_t fl = (MODE == 0 && !resid) ? bf[j] : (uint8_t)(BF_KEY | BF_VAL);
     const bool vprom = resid || (fl & BF_VAL);
-    const int ntok = resid ? sh.r : BLK;
-    const size_t tok0 = resid ? (size_t)sh.nb * BLK : (size_t)j * BLK;  // token index
+    const int ntok = resid ? rr : BLK;
+    const size_t tok0 = resid ? (size_t)nb * BLK : (size_t)j * BLK;  // token index
 
     // ---- logits ----
     if (MODE == 0 && tid == 0 && !resid) S.eta_b = t.eta[u * st.eta + j];  // overlaps the loads below

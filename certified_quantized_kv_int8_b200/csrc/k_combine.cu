@@ -61,7 +61,8 @@ __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_threshol
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = b * sh.Hkv + h / sh.G;
   const size_t row = (size_t)row_i;
-  const int nb = sh.nb;
+  int nb, r_unused;  // this batch row's sealed blocks
+  row_blocks(sh, b, nb, r_unused);
   const uint8_t* bf_g = sc.bflags + (size_t)unit * sh.nbm;
   const float* e8_g = sc.ell8 + row * sh.nbm;
   const float* e16_g = sc.ell16 + row * sh.nbm;
@@ -329,7 +330,7 @@ cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, cons
 cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
                           const Scratch& sc, cudaStream_t s) {
   // stage the head's keys and flags in shared memory up to 96 KiB
-  const size_t bytes = (size_t)sh.nb * 9;
+  const size_t bytes = (size_t)sh.nb_max * 9;
   const int staged = bytes <= 96u * 1024u ? 1 : 0;
   const int smem = staged ? (int)((bytes + 15) / 16 * 16) : 0;
   if (smem > 48 * 1024) {

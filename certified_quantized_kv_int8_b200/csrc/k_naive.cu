@@ -163,7 +163,7 @@ __device__ double naive_e_key(double dT, double dA, double m8T) {
 // zero for the next launch.
 template <int D, int G>
 __device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int nparts, int narr,
-                                   int unit,
+                                   int unit, int nb,
                                    size_t hrow0, float* __restrict__ out,
                                    float* __restrict__ e_key, float* __restrict__ e_val,
                                    uint8_t* __restrict__ rung, float* wsm, int* flag) {
@@ -232,7 +232,7 @@ __device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int
       const float* px = sc.part_x + (base + (size_t)(nparts - 1) * G + h) * 3;
       const float mr = __ldcg(px + 1);
       const double mres = mr == -INFINITY ? 0.0 : (double)__ldcg(px + 2) * exp((double)mr - M) / L;
-      const float ek = sh.nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
+      const float ek = nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
       e_key[row] = ek;
       e_val[row] = E / L;
       rung[row] = 0;
@@ -335,17 +335,20 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
   }
   if (tid < G) S.dmax[tid] = 0.f;  // published by the barrier before the first block
 
-  // work items: the nb sealed blocks, then the residual block (items nb and
-  // nb + 1 when it holds tokens); the nch CTAs of a unit take floor or ceil of
-  // items / nch consecutive items
+  // work items of the row: its nb sealed blocks, then the residual block
+  // (items nb and nb + 1 when it holds tokens); the nch CTAs of a unit take
+  // floor or ceil of items / nch consecutive items (none, in a row shorter
+  // than the grid's longest)
+  int nb, rr;
+  row_blocks(sh, b, nb, rr);
   const int nch = gridDim.x;
-  const int items = sh.nb + (sh.r > 0 ? 2 : 1);  // a residual block costs about two sealed ones
+  const int items = row_items(nb, rr);
   const int base = items / nch, rem = items - base * nch;
   const int i0 = chunk * base + min(chunk, rem);
   const int i1 = i0 + base + (chunk < rem ? 1 : 0);
   const int j0 = i0;
-  const int nblk = max(0, min(i1, sh.nb) - i0);
-  const bool do_res = i0 <= sh.nb && sh.nb < i1;  // the CTA holding item nb
+  const int nblk = max(0, min(i1, nb) - i0);
+  const bool do_res = i0 <= nb && nb < i1;  // the CTA holding item nb
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) mbar_init(&S.bar[s], 1);
     mbar_init_fence();
@@ -589,7 +592,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       for (int k2 = k; k2 <= hi; ++k2)
         mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
     }
-    naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, hrow0, out, e_key, e_val, rung,
+    naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, nb, hrow0, out, e_key, e_val, rung,
                              reinterpret_cast<float*>(dsm), &S.last);
     return;
   }
@@ -681,7 +684,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     const size_t rbase = ((size_t)unit * sc.max_chunks + nch) * G;
     float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK] base-2 logits, then weights
     float* mst = lg + G * BLK;                  // [G][2]
-    const int r = sh.r;
+    const int r = rr;
     const __half* kr = t.kres + u * st.res;
     const __half* vr = t.vres + u * st.res;
     constexpr int CPL = D / 32;
@@ -763,7 +766,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       sc.part_x[(rbase + tid) * 3 + 2] = mst[2 * tid + 1];
     }
   }
-  naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, hrow0, out, e_key, e_val, rung,
+  naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, nb, hrow0, out, e_key, e_val, rung,
                            reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::AT, &S.last);
 }
 
@@ -776,7 +779,7 @@ int naive_chunks(const DecodeShape& sh, int max_chunks) {
   if (per_unit > max_chunks - 1) per_unit = max_chunks - 1;  // one partial slot for the residual
   // at least 4 items per CTA: below that the per-CTA start-up and the merge of
   // more partials cost more than the parallelism gains (8K context: -10%)
-  if (per_unit > (sh.nb + 4) / 4) per_unit = (sh.nb + 4) / 4;
+  if (per_unit > (sh.nb_max + 4) / 4) per_unit = (sh.nb_max + 4) / 4;
   return per_unit < 1 ? 1 : per_unit;
 }
 

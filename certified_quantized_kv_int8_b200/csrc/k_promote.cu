@@ -56,8 +56,11 @@ __global__ void __launch_bounds__(THREADS) promote_kernel(Tier1 t, Strides st, i
   const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
   const size_t u = (size_t)unit0 + unit;
   const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
+  int nb, r_unused;
+  row_blocks(sh, b, nb, r_unused);
   const int j0 = blockIdx.x * sh.chunk_blocks;
-  const int j1 = min(sh.nb, j0 + sh.chunk_blocks);
+  const int j1 = min(nb, j0 + sh.chunk_blocks);
+  if (j0 >= j1) return;  // past the end of a shorter row
 
   bool headmask[G];
   bool any = MODE == 0;
@@ -173,7 +176,7 @@ cudaError_t launch_promote_t(const Tier1& t, const Strides& st, int unit0, const
 cudaError_t launch_promote(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                            const __half* q, const Scratch& sc, int mode, const __half* kstage,
                            int stage_nb, cudaStream_t s) {
-  if (sh.nb == 0) return cudaSuccess;
+  if (sh.nb_max == 0) return cudaSuccess;
 #define CQA_PROMOTE_CASE(DD, GG) \
   return launch_promote_t<DD, GG>(t, st, unit0, sh, q, sc, mode, kstage, stage_nb, s)
   if (sh.d == 128) {

@@ -120,17 +120,20 @@ __global__ void __launch_bounds__(NT, 5)
     S.qf[h][c] = __half2float(q[(hrow0 + h) * D + c]) * sh.sigma;
   }
 
-  // work items: the nb sealed blocks, then the residual block (items nb and
-  // nb + 1 when it holds tokens); the CTAs of a unit take floor or ceil of
-  // items / gridDim.x consecutive items
+  // work items of the row: its nb sealed blocks, then the residual block
+  // (items nb and nb + 1 when it holds tokens); the CTAs of a unit take floor
+  // or ceil of items / gridDim.x consecutive items (none, in a row shorter
+  // than the grid's longest)
+  int nb, rr;
+  row_blocks(sh, b, nb, rr);
   const int nch = gridDim.x;
-  const int items = sh.nb + (sh.r > 0 ? 2 : 1);  // a residual block costs about two sealed ones
+  const int items = row_items(nb, rr);
   const int base = items / nch, rem = items - base * nch;
   const int i0 = chunk * base + min(chunk, rem);
   const int i1 = i0 + base + (chunk < rem ? 1 : 0);
   const int j0 = i0;
-  const int nblk = max(0, min(i1, sh.nb) - i0);
-  const bool do_res = i0 <= sh.nb && sh.nb < i1;  // the CTA holding item nb
+  const int nblk = max(0, min(i1, nb) - i0);
+  const bool do_res = i0 <= nb && nb < i1;  // the CTA holding item nb
   if (tid == 0) {
     for (int s2 = 0; s2 < NST; ++s2) mbar_init(&S.bar[s2], 1);
     mbar_init_fence();
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(NT, 5)
   // the FP16 keys in device memory ----
   if (do_res) {
     float* lg = reinterpret_cast<float*>(dsm);  // [G][BLK]
-    const int r = sh.r;
+    const int r = rr;
     const __half* kr = t.kres + u * st.res;
     constexpr int CPL = D / 32;
     // four tokens per warp at a time: their key loads and the 4*G reductions are
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(NT, 5)
     for (int h = warp; h < G; h += NW) {
       const float x0 = lane < r ? lg[h * BLK + lane] : -INFINITY;
       const float x1 = lane + 32 < r ? lg[h * BLK + lane + 32] : -INFINITY;
-      float* lo = sc.logits + (hrow0 + h) * sc.ls + (size_t)sh.nb * BLK;
+      float* lo = sc.logits + (hrow0 + h) * sc.ls + (size_t)nb * BLK;
       if (lane < r) lo[lane] = x0;
       if (lane + 32 < r) lo[lane + 32] = x1;
       float lse = -INFINITY;
@@ -365,8 +368,7 @@ int score_chunks(const DecodeShape& sh) {
   const int units = sh.B * sh.Hkv;
   int per_unit = sh.sms * 5 / units;
   if (per_unit < 1) per_unit = 1;
-  const int items = sh.nb + (sh.r > 0 ? 2 : 1);
-  return per_unit < items ? per_unit : items;
+  return per_unit < sh.items_max ? per_unit : sh.items_max;
 }
 
 template <int D, int G>

@@ -148,17 +148,18 @@ __device__ double e_key_bound(double dT, double dA, double m8T) {
   return fmin(tanh(0.5 * dT), m_ub * expm1(2.0 * dT));
 }
 
-// dynamic shared memory: keys u64 [G][NP], mass f32 [G][nb], pflag u8 [nb], vflag u8 [nb]
+// dynamic shared memory, sized for the longest row (nbL = nb_max blocks):
+// keys u64 [G][NP], mass f32 [G][nbL], pflag u8 [nbL], vflag u8 [nbL]
 template <int G>
 __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, int unit0,
                                                          DecodeShape sh, cqa_thresholds th,
                                                          Scratch sc, int NP) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int nb = sh.nb;
+  const int nbL = sh.nb_max;
   uint64_t* keys_all = reinterpret_cast<uint64_t*>(smem);
   float* mass_all = reinterpret_cast<float*>(keys_all + (size_t)G * NP);
-  uint8_t* pflag = reinterpret_cast<uint8_t*>(mass_all + (size_t)G * nb);
-  uint8_t* vflag = pflag + nb;
+  uint8_t* pflag = reinterpret_cast<uint8_t*>(mass_all + (size_t)G * nbL);
+  uint8_t* vflag = pflag + nbL;
   constexpr int GT = THREADS / G;  // threads per head group
   __shared__ double slot_d[G][32];
   __shared__ float slot_f[G][32];
@@ -175,6 +176,8 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
   const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
   const int tid = threadIdx.x;
   const bool naive = th.naive != 0;
+  int nb, r_unused;  // this row's sealed blocks (at most nbL)
+  row_blocks(sh, b, nb, r_unused);
   Group grp;
   grp.id = tid / GT;
   grp.nthreads = GT;
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
   const int h = grp.id;  // this group's head
   const int tg = grp.tig;
   uint64_t* keys = keys_all + (size_t)h * NP;
-  float* mass = mass_all + (size_t)h * nb;
+  float* mass = mass_all + (size_t)h * nbL;
   const float* e8 = sc.ell8 + (hrow0 + h) * sh.nbm;
   const float* dl = sc.delta + (hrow0 + h) * sh.nbm;
 
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
       const float e = eta[j];
       uint8_t vp = 0;
       for (int hh = 0; hh < G; ++hh) {
-        if (mass_all[(size_t)hh * nb + j] * e > th.v_tol) {
+        if (mass_all[(size_t)hh * nbL + j] * e > th.v_tol) {
           vp = 1;
           atomicOr(&hf_s[hh], (unsigned)HF_VALUE);
         }
@@ -356,9 +359,9 @@ template <int G>
 cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                             const cqa_thresholds& th, const Scratch& sc, cudaStream_t s) {
   int NP = 2;
-  while (NP < sh.nb) NP <<= 1;
+  while (NP < sh.nb_max) NP <<= 1;
   if (NP < THREADS / G) NP = THREADS / G;  // at least one key per thread of a head group
-  const size_t smem = (size_t)G * NP * 8 + (size_t)G * sh.nb * 4 + 2 * (size_t)sh.nb;
+  const size_t smem = (size_t)G * NP * 8 + (size_t)G * sh.nb_max * 4 + 2 * (size_t)sh.nb_max;
   cudaError_t e = ensure_dynamic_smem((const void*)select_kernel<G>, (int)smem);
   if (e != cudaSuccess) return e;
   select_kernel<G><<<sh.B * sh.Hkv, THREADS, smem, s>>>(t, st, unit0, sh, th, sc, NP);

@@ -57,7 +57,9 @@ enum {
 
 typedef struct cqa_cache cqa_cache; /* opaque */
 
-/* Shape of one cache: every layer holds `batch` sequences of equal length. */
+/* Shape of one cache: every layer holds `batch` sequences.  Rows may hold
+ * different lengths (ragged batch): cqa_quantize_append_row grows one row,
+ * cqa_quantize_append grows every row by the same count. */
 typedef struct cqa_config {
   int32_t n_layers;
   int32_t batch;
@@ -88,7 +90,9 @@ typedef struct cqa_thresholds {
 } cqa_thresholds;
 
 /* Optional per-call diagnostics, all device pointers, any may be NULL.
- * nb = number of sealed 64-token blocks of the layer (length / 64). */
+ * nb = number of sealed 64-token blocks of the layer's longest row
+ * (length / 64); in a shorter row, entries past its own sealed blocks are
+ * unspecified. */
 typedef struct cqa_trace {
   int32_t* kstar;       /* [batch][n_q_heads] final K* after widening */
   uint8_t* block_flags; /* [batch][n_kv_heads][nb]: bit0 key promoted, bit1 value promoted */
@@ -109,10 +113,16 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out);
 /* Free everything the cache owns (synchronises the device first).  NULL is a no-op. */
 int cqa_cache_destroy(cqa_cache* cache);
 
-/* Tokens currently held by `layer` (host-side counter; no synchronisation). */
+/* Tokens currently held by `layer`: the longest batch row's length
+ * (host-side counter; no synchronisation). */
 int cqa_cache_length(const cqa_cache* cache, int layer, int32_t* out_len);
 
-/* Append n_new tokens to every batch row of `layer` (Methodology §1).
+/* Tokens held by each batch row of `layer`: out_lens is a host array of
+ * `batch` int32 (host-side counters; no synchronisation). */
+int cqa_cache_row_lengths(const cqa_cache* cache, int layer, int32_t* out_lens);
+
+/* Append n_new tokens to every batch row of `layer` (Methodology §1), each
+ * after its own row's tokens (rows of different lengths stay ragged).
  * k_fp16, v_fp16: device fp16 [batch][n_kv_heads][n_new][head_dim].
  * Every complete 64-token block is sealed: keys -> symmetric INT8 with one
  * fp32 scale per (block, channel) (s = amax/127, code = round-half-even(k/s)),
@@ -127,7 +137,16 @@ int cqa_cache_length(const cqa_cache* cache, int layer, int32_t* out_len);
 int cqa_quantize_append(cqa_cache* cache, int layer, const void* k_fp16, const void* v_fp16,
                         int n_new, void* stream);
 
-/* One certified decode step of `layer` for all batch rows (Methodology §2-§3).
+/* Append n_new tokens to batch row `row` of `layer` only, encoded exactly as
+ * cqa_quantize_append encodes them; the other rows keep their lengths.
+ * k_fp16, v_fp16: device fp16 [n_kv_heads][n_new][head_dim].
+ * CQA_ERR_INVALID_ARG if row is outside [0, batch); CQA_ERR_CAPACITY if the
+ * row's length + n_new > max_ctx.  n_new = 0 is a no-op. */
+int cqa_quantize_append_row(cqa_cache* cache, int layer, int row, const void* k_fp16,
+                            const void* v_fp16, int n_new, void* stream);
+
+/* One certified decode step of `layer` for all batch rows (Methodology §2-§3),
+ * each row over its own tokens (ragged rows allowed).
  * q_fp16: device fp16 [batch][n_q_heads][head_dim].
  * Outputs (device): out fp32 [batch][n_q_heads][head_dim]; e_key, e_val fp32
  * [batch][n_q_heads]; rung uint8 [batch][n_q_heads] = highest rung reached:
@@ -137,19 +156,22 @@ int cqa_quantize_append(cqa_cache* cache, int layer, const void* k_fp16, const v
  * max_c |out - O_dense| <= R_V * e_key + e_val, R_V = max_c (vmax_c - vmin_c)
  * of the head's kv head (exported by cqa_debug_export).
  * th: host pointer.  trace: host pointer to a cqa_trace, or NULL.
- * CQA_ERR_EMPTY if the layer holds no token. */
+ * CQA_ERR_EMPTY if some batch row of the layer holds no token. */
 int cqa_decode(cqa_cache* cache, int layer, const void* q_fp16, const cqa_thresholds* th,
                float* out, float* e_key, float* e_val, uint8_t* rung, const cqa_trace* trace,
                void* stream);
 
 /* Exact attention softmax(q K^T / sqrt(head_dim)) V of `layer` over the FP16
  * originals (Tier 2 plus the residual block), fp32 accumulation: the O_dense
- * the fallback ladder returns.  q_fp16 and out as in cqa_decode. */
+ * the fallback ladder returns.  q_fp16 and out as in cqa_decode, each row
+ * over its own tokens; CQA_ERR_EMPTY if some row holds no token. */
 int cqa_dense_reference(cqa_cache* cache, int layer, const void* q_fp16, float* out, void* stream);
 
 /* Copy one Tier-1 array of `layer` to host memory (synchronous; for tests and
  * inspection).  `what` selects the array, laid out as stated, with nb the
- * layer's sealed block count and d = head_dim:
+ * layer's sealed block count and d = head_dim.  In a ragged layer each
+ * (batch row, kv head) takes its own row's extent (its nb, length % 64 and
+ * length), and the units follow one another in [batch][n_kv_heads] order:
  *   CQA_EXPORT_KCODES   int8  [batch][n_kv_heads][nb][64][d]
  *   CQA_EXPORT_KSCALE   fp32  [batch][n_kv_heads][nb][d]
  *   CQA_EXPORT_VCODES   uint8 [batch][n_kv_heads][nb][64][d/2]  (channel 2j low nibble)

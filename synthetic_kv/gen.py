@@ -115,6 +115,7 @@ class Workload:
     tie_logit: float = 6.0
     tie_jitter: float = 0.02
     tie_layer_all: int = 17  # layer whose every kv group gets near-tie blocks
+    row_ctx: tuple = ()  # ragged batch: tokens of each batch row (ctx = the longest)
     extra: dict = field(default_factory=dict, compare=False, hash=False)
 
     @property
@@ -137,7 +138,16 @@ WORKLOADS = {
         value_dist="student_t3"),
     "llama8b_128k_needle": Workload(
         "llama8b_128k_needle", 32, 1, 32, 8, 128, 131072, 4, 10.0, needle=True),
+    # a ragged batch: four rows of different lengths, the longest 32K
+    "llama8b_ragged_b4": Workload(
+        "llama8b_ragged_b4", 32, 4, 32, 8, 128, 32768, 4, 10.0,
+        row_ctx=(32768, 4096 + 37, 16384 + 5, 8192)),
 }
+
+
+def row_lengths(w: Workload) -> list[int]:
+    """Tokens of each batch row when timing starts."""
+    return list(w.row_ctx) if w.row_ctx else [w.ctx] * w.batch
 
 
 def default_thresholds(w: Workload) -> dict:
@@ -269,6 +279,12 @@ def _plant(w, layer, b, kvh, t0, t1, k, device):
             val = ct * qbar[None, :] + 0.3 * base + w.tie_jitter * jit
             k[lo - t0:hi - t0] = val.float().half()
     return k
+
+
+def kv_row(w: Workload, layer: int, b: int, t0: int, t1: int, device="cpu"):
+    """Keys and values of one batch row: float16 [n_kv_heads][t1 - t0][head_dim]."""
+    ks, vs = zip(*(kv_unit(w, layer, b, g, t0, t1, device) for g in range(w.n_kv_heads)))
+    return torch.stack(ks).contiguous(), torch.stack(vs).contiguous()
 
 
 def kv_layer(w: Workload, layer: int, t0: int, t1: int, device="cpu"):

@@ -192,5 +192,15 @@ def run_decode(cache, layer, q, th, stream=None):
     return {k: v.cpu().numpy() for k, v in res.items()}
 
 
-def row(res, b):
-    return {k: v[b] for k, v in res.items()}
+_BLOCK_AXIS = ("block_flags", "ell8", "ell16", "delta")
+
+
+def row(res, b, nb=None):
+    """Batch row b of run_decode's result; with nb, the per-block trace arrays are
+    cut to the row's own nb sealed blocks (a ragged batch sizes them for its
+    longest row)."""
+    out = {k: v[b] for k, v in res.items()}
+    if nb is not None:
+        for k in _BLOCK_AXIS:
+            out[k] = out[k][:, :nb]
+    return out

@@ -71,3 +71,28 @@ def test_cpu_baseline_reports_threads_and_single_thread():
     d = bench.cpu_baseline(w, th, budget_s=1.0)
     assert d["kind"] == "oracle" and d["value"] > 0 and d["cores"] >= 1
     assert d["single_thread_value"] > 0
+
+
+def test_ragged_oracle_scaling():
+    """The oracle's sampled row stands for the step's rows in proportion to length."""
+    import dataclasses
+    import synthetic_kv as sk
+    w = sk.WORKLOADS["llama8b_ragged_b4"]
+    assert bench.rows_per_sample(w) == pytest.approx(sum(w.row_ctx) / w.row_ctx[0])
+    u = dataclasses.replace(sk.WORKLOADS["tiny"], batch=3)
+    assert bench.rows_per_sample(u) == 3
+
+
+def test_reference_arm_on_a_ragged_batch(capsys):
+    import dataclasses
+    import synthetic_kv as sk
+    w = dataclasses.replace(sk.WORKLOADS["tiny"], batch=2, row_ctx=(1024, 300))
+    sk.WORKLOADS["tiny_ragged_test"] = dataclasses.replace(w, name="tiny_ragged_test")
+    try:
+        rc = bench.main(["--impl", "reference", "--workload", "tiny_ragged_test", "--steps", "1",
+                         "--warmup", "3"])
+    finally:
+        del sk.WORKLOADS["tiny_ragged_test"]
+    assert rc == 0
+    d = json.loads([l for l in capsys.readouterr().out.splitlines() if l.strip()][0])
+    assert d["config"]["row_ctx"] == [1024, 300] and d["value"] > 0

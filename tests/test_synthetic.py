@@ -41,3 +41,17 @@ def test_student_t_values_and_drift():
     F1, _ = sk.kv_unit(flat, 0, 0, 0, 32768 - 64, 32768)
     drift = (K1.double() - F1.double()).mean(0)
     assert float(drift.abs().mean()) > 0.5  # near beta * |u| at the end of the context
+
+
+def test_ragged_rows():
+    """A ragged workload lists each row's length; kv_row is the row's kv_unit stack."""
+    w = sk.WORKLOADS["llama8b_ragged_b4"]
+    lens = sk.row_lengths(w)
+    assert len(lens) == w.batch and max(lens) == w.ctx and len(set(lens)) == w.batch
+    assert sk.row_lengths(sk.WORKLOADS["tiny"]) == [1024]
+    t = sk.WORKLOADS["tiny"]
+    K, V = sk.kv_row(t, 0, 0, 10, 30)
+    assert K.shape == (t.n_kv_heads, 20, t.head_dim) and K.is_contiguous()
+    for g in range(t.n_kv_heads):
+        k, v = sk.kv_unit(t, 0, 0, g, 10, 30)
+        assert torch.equal(K[g], k) and torch.equal(V[g], v)
