@@ -99,7 +99,10 @@ void chunking(int units, int nb, int sms, int* chunk_blocks, int* nchunks) {
   *nchunks = nc < 1 ? 1 : nc;
 }
 
-int max_chunks_for(int units, int sms) { return (target_ctas(sms) + units - 1) / units + 1; }
+// Partial slots per unit: the CTAs one unit may receive (a whole grid's worth
+// split over one row's kv heads, when the other rows of a ragged batch are
+// short) plus the residual block's slot.
+int max_chunks_for(int Hkv, int sms) { return target_ctas(sms) / Hkv + 2; }
 
 const int32_t* row_lens(const cqa_cache* c, int layer) {
   return c->len + (size_t)layer * c->cfg.batch;
@@ -128,15 +131,16 @@ DecodeShape shape_of(const cqa_cache* c, int layer) {
   sh.G = c->G;
   sh.d = c->cfg.head_dim;
   sh.nb_max = 0;
-  sh.items_max = 1;
+  sh.items_sum = 0;
   const int32_t* L = row_lens(c, layer);
   for (int b = 0; b < sh.B; ++b) {
     const int nb = L[b] / BLK, r = L[b] - (L[b] / BLK) * BLK;
     if (nb > sh.nb_max) sh.nb_max = nb;
-    if (row_items(nb, r) > sh.items_max) sh.items_max = row_items(nb, r);
+    sh.items_sum += (long long)sh.Hkv * row_items(nb, r);
   }
   sh.nbm = c->nbm;
   sh.lens = c->lens_dev + (size_t)layer * sh.B;
+  sh.lens_host = L;
   sh.sigma = (float)(1.0 / sqrt((double)sh.d));
   sh.sms = c->sms;
   chunking(sh.B * sh.Hkv, sh.nb_max, sh.sms, &sh.chunk_blocks, &sh.nchunks);
@@ -325,7 +329,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
     return CQA_ERR_CUDA;
   }
   cc->sms = sms;
-  const size_t max_chunks = (size_t)max_chunks_for(c.batch * c.n_kv_heads, sms);
+  const size_t max_chunks = (size_t)max_chunks_for(c.n_kv_heads, sms);
 
   // one device allocation, carved into aligned pieces
   size_t off = 0;

@@ -96,9 +96,10 @@ struct Scratch {
 // length of its own row from `lens`.
 struct DecodeShape {
   int B, Hq, Hkv, G, d, nb_max, nbm, nchunks, chunk_blocks;
-  int items_max;        // max over rows of the streaming passes' work items (see row_items)
+  long long items_sum;  // sum over (row, kv head) units of their work items
   int sms;              // streaming multiprocessors of the cache's device (grid sizing)
   const int32_t* lens;  // device [B]: tokens held by each batch row of the layer
+  const int32_t* lens_host;  // the same lengths in host memory (grid sizing by launchers)
   float sigma;
 };
 
@@ -112,6 +113,17 @@ __device__ __forceinline__ void row_blocks(const DecodeShape& sh, int b, int& nb
 // Work items of a row in the streaming passes: its sealed blocks, then the
 // residual block, which costs about two sealed ones when it holds tokens.
 __host__ __device__ __forceinline__ int row_items(int nb, int r) { return nb + (r > 0 ? 2 : 1); }
+
+// CTAs per (row, kv head) unit of a streaming pass whose grid targets `target`
+// resident CTAs: units receive CTAs in proportion to their work items, so the
+// rows of a ragged batch finish together; at most `cap`, at least one.  The
+// host sizes the grid with the same integer arithmetic.
+__host__ __device__ __forceinline__ int unit_ctas(int target, int items, long long items_sum,
+                                                  int cap) {
+  long long n = (long long)target * items / (items_sum > 0 ? items_sum : 1);
+  if (n > cap) n = cap;
+  return n < 1 ? 1 : (int)n;
+}
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
 // again only when a launch needs more than already granted: the attribute

@@ -50,6 +50,16 @@ constexpr int NST = 3;         // stages per CTA
 constexpr int TPW = BLK / NW;  // tokens of each block handled by one warp
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
+constexpr int NAIVE_CTAS_PER_SM = 4;  // grid target: resident CTAs per SM
+
+// Most CTAs one unit with nb sealed blocks takes: one partial slot stays for
+// the residual block, and each CTA gets at least 4 items (below that the
+// per-CTA start-up and the merge of more partials cost more than the
+// parallelism gains: 8K context, -10%).
+__host__ __device__ __forceinline__ int naive_cap(int nb, int max_chunks) {
+  const int c = (nb + 4) / 4;
+  return c < max_chunks - 1 ? c : max_chunks - 1;
+}
 
 template <int D>
 struct NaiveLayout {
@@ -337,12 +347,14 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 
   // work items of the row: its nb sealed blocks, then the residual block
   // (items nb and nb + 1 when it holds tokens); the nch CTAs of a unit take
-  // floor or ceil of items / nch consecutive items (none, in a row shorter
-  // than the grid's longest)
+  // floor or ceil of items / nch consecutive items
   int nb, rr;
   row_blocks(sh, b, nb, rr);
-  const int nch = gridDim.x;
   const int items = row_items(nb, rr);
+  // this unit's CTAs: its share of the grid target in proportion to its items
+  const int nch = min((int)gridDim.x, unit_ctas(sh.sms * NAIVE_CTAS_PER_SM, items, sh.items_sum,
+                                                naive_cap(nb, sc.max_chunks)));
+  if (chunk >= nch) return;  // a unit of a shorter row has fewer CTAs than the grid's width
   const int base = items / nch, rem = items - base * nch;
   const int i0 = chunk * base + min(chunk, rem);
   const int i1 = i0 + base + (chunk < rem ? 1 : 0);
@@ -770,17 +782,20 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
                            reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::AT, &S.last);
 }
 
-// CTAs per unit of the streaming pass: four resident CTAs per SM hold the
-// whole grid (one wave), so the unit's last arrival is never a CTA that
-// waited for a free slot
+// Grid width of the streaming pass: the most CTAs any unit receives.  Units
+// share sms * 4 CTAs (four resident per SM hold the whole grid, one wave, so a
+// unit's last arrival is never a CTA that waited for a free slot) in
+// proportion to their work items; units of shorter rows leave the rest of
+// their grid row empty.
 int naive_chunks(const DecodeShape& sh, int max_chunks) {
-  const int units = sh.B * sh.Hkv;
-  int per_unit = sh.sms * 4 / units;
-  if (per_unit > max_chunks - 1) per_unit = max_chunks - 1;  // one partial slot for the residual
-  // at least 4 items per CTA: below that the per-CTA start-up and the merge of
-  // more partials cost more than the parallelism gains (8K context: -10%)
-  if (per_unit > (sh.nb_max + 4) / 4) per_unit = (sh.nb_max + 4) / 4;
-  return per_unit < 1 ? 1 : per_unit;
+  int w = 1;
+  for (int b = 0; b < sh.B; ++b) {
+    const int T = sh.lens_host[b], nb = T / BLK, items = row_items(nb, T - nb * BLK);
+    const int n = unit_ctas(sh.sms * NAIVE_CTAS_PER_SM, items, sh.items_sum,
+                            naive_cap(nb, max_chunks));
+    w = n > w ? n : w;
+  }
+  return w;
 }
 
 template <int D, int G>

@@ -42,6 +42,7 @@ constexpr int TPW = BLK / NW;  // tokens of each block scored by one warp
 constexpr int CH = 8;          // channels per lane
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
+constexpr int SCORE_CTAS_PER_SM = 5;  // grid target: resident CTAs per SM
 
 template <int D>
 struct ScoreLayout {
@@ -121,13 +122,15 @@ __global__ void __launch_bounds__(NT, 5)
   }
 
   // work items of the row: its nb sealed blocks, then the residual block
-  // (items nb and nb + 1 when it holds tokens); the CTAs of a unit take floor
-  // or ceil of items / gridDim.x consecutive items (none, in a row shorter
-  // than the grid's longest)
+  // (items nb and nb + 1 when it holds tokens); the nch CTAs of a unit take
+  // floor or ceil of items / nch consecutive items
   int nb, rr;
   row_blocks(sh, b, nb, rr);
-  const int nch = gridDim.x;
   const int items = row_items(nb, rr);
+  // this unit's CTAs: its share of the grid target in proportion to its items
+  const int nch =
+      min((int)gridDim.x, unit_ctas(sh.sms * SCORE_CTAS_PER_SM, items, sh.items_sum, items));
+  if (chunk >= nch) return;  // a unit of a shorter row has fewer CTAs than the grid's width
   const int base = items / nch, rem = items - base * nch;
   const int i0 = chunk * base + min(chunk, rem);
   const int i1 = i0 + base + (chunk < rem ? 1 : 0);
@@ -363,12 +366,17 @@ __global__ void __launch_bounds__(NT, 5)
   }
 }
 
-// CTAs per unit: five resident CTAs per SM hold the whole grid (one wave)
+// Grid width: the most CTAs any unit receives.  Units share sms * 5 CTAs (five
+// resident per SM hold the whole grid, one wave) in proportion to their work
+// items, at most one CTA per item.
 int score_chunks(const DecodeShape& sh) {
-  const int units = sh.B * sh.Hkv;
-  int per_unit = sh.sms * 5 / units;
-  if (per_unit < 1) per_unit = 1;
-  return per_unit < sh.items_max ? per_unit : sh.items_max;
+  int w = 1;
+  for (int b = 0; b < sh.B; ++b) {
+    const int T = sh.lens_host[b], nb = T / BLK, items = row_items(nb, T - nb * BLK);
+    const int n = unit_ctas(sh.sms * SCORE_CTAS_PER_SM, items, sh.items_sum, items);
+    w = n > w ? n : w;
+  }
+  return w;
 }
 
 template <int D, int G>
