@@ -12,8 +12,10 @@
 //
 // One CTA streams a chunk of consecutive blocks of one (batch row, kv head)
 // through a ring of NST shared-memory stages filled by bulk copies (INT8
-// codes, key scales, INT4 codes, value scale/offset of one block per stage):
-// 14.5 KiB per block for head_dim 128, every byte of Tier 1 read once.
+// codes, key scales, INT4 codes, value scale/offset and the 16 aligned bytes
+// of eta holding eta_b, of one block per stage): 14.5 KiB per block for
+// head_dim 128, every byte of Tier 1 read once.  The issuing thread never
+// waits for a load of its own, so the copies leave as soon as a stage frees.
 //
 // The pass is bound by instruction issue and the FP32 pipe rather than by HBM
 // (per token and kv head: 128 INT8 and 128 INT4 conversions and 2*G*head_dim
@@ -154,7 +156,7 @@ struct NaiveSmem {
   float alpha[NW][G];              // rescale factor of each warp's running state
   float ellp[2][NW][G];            // trace: log2-sum-exp of each warp's tokens of a block
   float dmax[G];
-  float eta[NST];  // eta_b of the block held by each stage
+  __align__(16) float eta[NST][4];  // the 16-byte run of eta holding eta_b of each stage's block
   int last;        // this CTA merges its unit's partials
   uint64_t bar[NST];
 };
@@ -372,8 +374,9 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     const int j = j0 + k;
     unsigned char* dst = dsm + (size_t)(k % NST) * LY::STAGE;
     uint64_t* bar = &S.bar[k % NST];
-    S.eta[k % NST] = t.eta[u * st.eta + j];  // read by consumers after the stage's barrier
-    mbar_arrive_expect_tx(bar, LY::STAGE);
+    const size_t ei = u * st.eta + j;  // eta_b arrives with the block: 16 aligned bytes holding it
+    mbar_arrive_expect_tx(bar, LY::STAGE + 16);
+    bulk_g2s(&S.eta[k % NST][0], t.eta + (ei & ~(size_t)3), 16, bar);
     bulk_g2s(dst, t.kcodes + u * st.kcodes + (size_t)j * LY::KB, LY::KB, bar);
     bulk_g2s(dst + LY::KB, t.kscale + u * st.kscale + (size_t)j * D, LY::SB, bar);
     bulk_g2s(dst + LY::KB + LY::SB, t.vcodes + u * st.vcodes + (size_t)j * LY::VB, LY::VB, bar);
@@ -529,7 +532,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 #pragma unroll
     for (int m = CPT; m < 32; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
     lrun = fmaf(lrun, alpha, ps);
-    erun = fmaf(erun, alpha, S.eta[stg] * ps);
+    erun = fmaf(erun, alpha, S.eta[stg][(u * st.eta + j) & 3] * ps);
     mrun = mnew;
     if (trace) {
       float es = 0.f;
