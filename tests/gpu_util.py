@@ -163,8 +163,14 @@ def compare_decode(gpu, ora, th, G, log: TieLog, label=""):
                 v = np.sort(key[P])[::-1][: r + 1]
                 if v.size > 1 and np.min(np.abs(np.diff(v))) <= TIE * max(1.0, np.abs(v).max()):
                     tie = True
-            layer_level = (rg == 4) != (ro == 4) and any(
-                e[1].get("label") == label for e in log.entries)
+            # a whole-layer (rung 4) difference is excused only when a tie was
+            # logged for this same (layer, batch row) and the oracle's count of
+            # rung-3 heads sits within one head of the trigger, so that one
+            # tied head could have moved it across
+            n3 = int(sum(int(np.sum(gg["key_fail"] | gg["rank_fail"])) for gg in groups))
+            need = math.ceil(th.layer_dense_frac * Hq)
+            layer_level = ((rg == 4) != (ro == 4) and abs(n3 - need) <= 1 and any(
+                e[1].get("label") == label for e in log.entries))
             if not tie and not layer_level:
                 raise AssertionError(f"{label} head {h}: rung {rg} vs oracle {ro}")
             log.add("rung", label=label, head=h, gpu=rg, oracle=ro)

@@ -115,3 +115,40 @@ def test_bounds_hold_on_decoded_heads(rng, tau, heavy_v):
                 # value part alone: same weights, exact vs reconstructed values
                 v_exact = g["p"][h] @ u["V"].astype(np.float64)
                 assert np.abs(v_exact - res["out"][hq]).max() <= res["e_val"][hq] + 1e-9
+
+
+def _eval_fixture_unit():
+    """The unit of tests/golden/eval_hand.txt: three sealed blocks and ten residual tokens."""
+    d, T = 64, 3 * BLOCK + 10
+    K = np.zeros((T, d), np.float16)
+    K[64:128, 0] = 1.0
+    K[128, 0] = -100.0
+    K[129:192, 0] = 0.5
+    K[192:, 0] = 1.5
+    V = np.zeros((T, d), np.float16)
+    V[:, 1] = 15.0
+    V[0, 2], V[64, 2], V[130, 2] = 0.5, 0.25, 0.125
+    q = np.zeros((1, d), np.float16)
+    q[0, 0] = 8.0
+    return q, build_unit(K, V)
+
+
+@pytest.mark.parametrize("case", ["A", "B"])
+def test_e_val_hand_fixture(case):
+    """E_val = sum over INT4-valued blocks of final attention mass x eta_b, against
+    the hand-worked closed form (value-promoted blocks excluded; the mass is the
+    final mixed distribution, residual included, not the INT8 estimate)."""
+    from oracle.cqa_oracle import decode_group
+    g = load("eval_hand.txt")
+    q, u = _eval_fixture_unit()
+    np.testing.assert_array_equal(u["eta"], g["eta"].astype(np.float32))
+    assert float(u["kscale"][2, 0]) == float(g["s_block2"][0])
+    if case == "A":
+        th = Thresholds(tau_cov=1.0, v_tol=float(g["v_tol"][0]))
+    else:
+        th = Thresholds(tau_cov=0.5, eps_key=1.0, v_tol=float(g["v_tol"][0]))
+    res = decode_group(q, u, th)
+    np.testing.assert_array_equal(res["P"], g[f"promoted_{case}"].astype(bool))
+    np.testing.assert_array_equal(res["VP"], g["value_promoted"].astype(bool))
+    want = float(g[f"e_val_{case}"][0])
+    assert abs(float(res["e_val"][0]) - want) <= 1e-13 * want
