@@ -61,7 +61,8 @@ class _Thresholds(ctypes.Structure):
     _fields_ = [("tau_cov", ctypes.c_float), ("eps_key", ctypes.c_float),
                 ("max_expand", ctypes.c_int32), ("v_tol", ctypes.c_float),
                 ("rank_r", ctypes.c_int32), ("eps_val", ctypes.c_float),
-                ("layer_dense_frac", ctypes.c_float), ("naive", ctypes.c_int32)]
+                ("layer_dense_frac", ctypes.c_float), ("naive", ctypes.c_int32),
+                ("rank_tol", ctypes.c_int32)]
 
 
 class _Trace(ctypes.Structure):
@@ -79,15 +80,16 @@ class Thresholds:
     eps_key: float = 5e-3
     max_expand: int = 4
     v_tol: float = 0.05
-    rank_r: int = 4
+    rank_r: int = 8
     eps_val: float = float("inf")
     layer_dense_frac: float = 0.5
     naive: bool = False
+    rank_tol: int = 2
 
     def as_c(self) -> _Thresholds:
         return _Thresholds(self.tau_cov, self.eps_key, int(self.max_expand), self.v_tol,
                            int(self.rank_r), self.eps_val, self.layer_dense_frac,
-                           1 if self.naive else 0)
+                           1 if self.naive else 0, int(self.rank_tol))
 
     def float32_rounded(self) -> dict:
         """The values the library sees (floats rounded to float32), as a dict."""

@@ -610,7 +610,8 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
     return CQA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return CQA_ERR_INVALID_ARG;
   const cqa_thresholds tv = *th;
-  if (!(tv.tau_cov >= 0.f) || tv.max_expand < 0 || tv.rank_r < 0 || isnan(tv.eps_key) ||
+  if (!(tv.tau_cov >= 0.f) || tv.max_expand < 0 || tv.rank_r < 0 ||
+      tv.rank_r > CQA_MAX_RANK_R || tv.rank_tol < 0 || isnan(tv.eps_key) ||
       isnan(tv.v_tol) || isnan(tv.eps_val) || isnan(tv.layer_dense_frac))
     return CQA_ERR_INVALID_ARG;
   if (min_len(cc, layer) == 0) return CQA_ERR_EMPTY;

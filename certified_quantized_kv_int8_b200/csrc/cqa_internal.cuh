@@ -22,6 +22,7 @@ namespace cqa {
 
 constexpr int BLK = 64;  // tokens per block
 constexpr int VG = 32;   // channels per INT4 value group
+constexpr int MAX_RANK_R = CQA_MAX_RANK_R;  // longest top-r list of the rank check
 
 // bits of the per-block flag byte
 constexpr uint8_t BF_KEY = 1;  // FP16 keys promoted

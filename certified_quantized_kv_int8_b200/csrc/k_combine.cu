@@ -8,12 +8,15 @@
 // with their FP16 ranking, a mismatch sends the head to dense attention;
 // rung 4 recomputes the whole layer densely).
 //
-// Readings used: the check compares the ordered top-min(rank_r, |P|) lists of
-// promoted blocks by INT8 and by FP16 block log-mass (ties to the lower block
-// index); rung 3 also fires when E_key stayed above eps_key after widening;
-// rung 4 fires when at least need_dense = ceil(layer_dense_frac * n_q_heads)
-// heads of a (layer, batch row) took rung 3 that way.  After the attention
-// pass, a head whose E_val exceeds eps_val also takes rung 3 (post-check).
+// Readings used: the check takes the top-min(rank_r, |P|) promoted blocks by
+// INT8 and by FP16 block log-mass (each ordered by log-mass descending, ties
+// to the lower block index) and counts the pairs of the union of the two lists
+// that the two rankings order the other way round; more than rank_tol such
+// pairs is a failure (rank_tol = 0: the ordered lists must be equal).  Rung 3
+// also fires when E_key stayed above eps_key after widening; rung 4 fires when
+// at least need_dense = ceil(layer_dense_frac * n_q_heads) heads of a (layer,
+// batch row) took rung 3 that way.  After the attention pass, a head whose
+// E_val exceeds eps_val also takes rung 3 (post-check, not counted for rung 4).
 #include "cqa_internal.cuh"
 
 namespace cqa {
@@ -31,9 +34,11 @@ __device__ __forceinline__ bool before(KI a, KI b) { return a.k > b.k || (a.k ==
 // Rank check and the rung 3 / rung 4 decision, before the attention pass.
 // One CTA of DT threads per (batch row, query head).  The head's INT8 and FP16
 // block log-masses and the block flags are staged in shared memory when they
-// fit (else read in place); the ordered top-r lists are then built one rank
-// at a time by a CTA-wide arg-best under the (key desc, index asc) order.  The
-// last CTA of a batch row to finish takes the whole-layer decision (rung 4).
+// fit (else read in place).  The two top-r lists are built one rank at a time
+// by CTA-wide arg-bests under the (key desc, index asc) orders; their union U
+// (at most 2 * MAX_RANK_R blocks) is then compared pair by pair, one pair per
+// thread per round.  The last CTA of a batch row to finish takes the
+// whole-layer decision (rung 4).
 constexpr int DT = 256;
 constexpr int DW = DT / 32;
 
@@ -55,6 +60,9 @@ __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_threshol
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ KI red[2][DW];
   __shared__ int cnt[DW];
+  __shared__ int top8[MAX_RANK_R], top16[MAX_RANK_R];
+  __shared__ int uni[2 * MAX_RANK_R];
+  __shared__ int nuni;
   __shared__ int flag;
   const int row_i = blockIdx.x;  // b * Hq + h
   const int b = row_i / sh.Hq, h = row_i - b * sh.Hq;
@@ -93,10 +101,10 @@ __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_threshol
   np = 0;
 #pragma unroll
   for (int w = 0; w < DW; ++w) np += cnt[w];
-  const int r = min(th.rank_r, np);
+  const int r = min(min(th.rank_r, MAX_RANK_R), np);
+  // the two top-r lists
   KI p8{INFINITY, -1}, p16{INFINITY, -1};
-  bool fail = false;
-  for (int k = 0; k < r && !fail; ++k) {
+  for (int k = 0; k < r; ++k) {
     KI c8{-INFINITY, 0x7fffffff}, c16{-INFINITY, 0x7fffffff};
     for (int j = tid; j < nb; j += DT) {
       if (!(bf[j] & BF_KEY)) continue;
@@ -121,8 +129,50 @@ __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_threshol
     }
     p8 = c8;
     p16 = c16;
-    fail = p8.i != p16.i;  // the same on every thread
+    if (tid == 0) {
+      top8[k] = p8.i;
+      top16[k] = p16.i;
+    }
   }
+  __syncthreads();
+  // union: the INT8 list, then the FP16 entries it does not hold (warp 0)
+  if (warp == 0) {
+    int base = r;
+    for (int k0 = 0; k0 < r; k0 += 32) {
+      const int k = k0 + lane;
+      bool fresh = false;
+      if (k < r) {
+        fresh = true;
+        for (int i = 0; i < r; ++i) fresh &= top8[i] != top16[k];
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, fresh);
+      if (fresh) uni[base + __popc(m & ((1u << lane) - 1u))] = top16[k];
+      base += __popc(m);
+    }
+    for (int k = lane; k < r; k += 32) uni[k] = top8[k];
+    if (lane == 0) nuni = base;
+  }
+  __syncthreads();
+  // discordant pairs of U: the two orders place the pair the other way round
+  const int nu = nuni;
+  int disc = 0;
+  for (int pi = tid; pi < nu * nu; pi += DT) {
+    const int i = pi / nu, j = pi - i * nu;
+    if (i >= j) continue;
+    const int a = uni[i], c = uni[j];
+    const bool a8 = before(KI{e8[a], a}, KI{e8[c], c});
+    const bool a16 = before(KI{e16[a], a}, KI{e16[c], c});
+    disc += a8 != a16 ? 1 : 0;
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) disc += __shfl_xor_sync(0xffffffffu, disc, m);
+  __syncthreads();  // cnt was read above
+  if (lane == 0) cnt[warp] = disc;
+  __syncthreads();
+  disc = 0;
+#pragma unroll
+  for (int w = 0; w < DW; ++w) disc += cnt[w];
+  const bool fail = disc > th.rank_tol;
   const bool naive = th.naive != 0;
   if (tid == 0) {
     uint8_t hf = sc.hflags[row];

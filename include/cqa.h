@@ -70,6 +70,9 @@ typedef struct cqa_config {
   int32_t device;     /* CUDA device ordinal the cache lives on */
 } cqa_config;
 
+/* Largest rank_r a decode accepts (CQA_ERR_INVALID_ARG above it). */
+#define CQA_MAX_RANK_R 64
+
 /* Runtime thresholds of one decode call (Methodology §3).  tau_cov and v_tol
  * are named by the method; the other fields are this library's readings of
  * triggers the method leaves unstated. */
@@ -80,13 +83,19 @@ typedef struct cqa_thresholds {
   int32_t max_expand;     /* ... at most max_expand times; still above -> rung 3 */
   float v_tol;            /* rung 2: FP16 values for block b if some head's
                              m8_b * eta_b > v_tol (m8 = INT8-estimated block mass) */
-  int32_t rank_r;         /* rank check: ordered top-min(rank_r, |P|) promoted blocks by
-                             INT8 and by FP16 log-mass must agree, else rung 3 */
+  int32_t rank_r;         /* rank check (Methodology §3, rank-consistency check): over the
+                             promoted blocks, the top-min(rank_r, |P|) blocks by INT8 and by
+                             FP16 block log-mass (ties to the lower block index) form a union
+                             U; the rankings disagree when more than rank_tol pairs of U are
+                             ordered the other way round by the two log-masses -> rung 3.
+                             0 <= rank_r <= CQA_MAX_RANK_R; 0 disables the check */
   float eps_val;          /* rung 3 also when E_val > eps_val (+inf disables) */
   float layer_dense_frac; /* rung 4 when >= ceil(layer_dense_frac * n_q_heads) heads of a
-                             (layer, batch row) took rung 3 */
+                             (layer, batch row) took rung 3 by the rank check or by E_key */
   int32_t naive;          /* 1: certification off (no promotion, no ladder; bounds still
                              reported; one fused INT8/INT4 streaming pass), 0: certified */
+  int32_t rank_tol;       /* discordant pairs of U the rank check tolerates (>= 0); 0 makes
+                             it require equal ordered top-r lists */
 } cqa_thresholds;
 
 /* Optional per-call diagnostics, all device pointers, any may be NULL.

@@ -19,6 +19,7 @@ from .cqa_oracle import (  # noqa: F401
     e_key_bound,
     coverage_kstar,
     rank_consistent,
+    rank_discordance,
     decode,
     Thresholds,
 )

@@ -192,7 +192,7 @@ def coverage_kstar(ell8: np.ndarray, m8: np.ndarray, m_res: float, tau_cov: floa
 @dataclass
 class Thresholds:
     """Runtime thresholds.  tau_cov (coverage) and v_tol (value tolerance) are
-    named by the method; eps_key, eps_val, rank_r, max_expand and
+    named by the method; eps_key, eps_val, rank_r, rank_tol, max_expand and
     layer_dense_frac are this implementation's readings of the ladder's
     unstated triggers."""
 
@@ -200,7 +200,8 @@ class Thresholds:
     eps_key: float = 5e-3
     eps_val: float = float("inf")
     v_tol: float = 0.05
-    rank_r: int = 4
+    rank_r: int = 8
+    rank_tol: int = 2
     max_expand: int = 4
     layer_dense_frac: float = 0.5
     naive: bool = False  # certification off: no promotion, no ladder
@@ -228,17 +229,47 @@ def _top_r(keys: np.ndarray, idx: np.ndarray, r: int) -> list:
     return [int(idx[i]) for i in o[:r]]
 
 
-def rank_consistent(ell8: np.ndarray, ell16: np.ndarray, promoted: np.ndarray, rank_r: int) -> bool:
-    """Block-ranking consistency check (Methodology §3): over the promoted blocks,
-    the ordered top-r list by INT8 block log-mass must equal the ordered top-r
-    list by FP16 block log-mass, r = min(rank_r, number promoted), ties to the
-    lower block index.  The pages name the check, not its exact form; this is
-    the reading used here (parity unpinned beyond this stated rule)."""
+def rank_discordance(ell8: np.ndarray, ell16: np.ndarray, promoted: np.ndarray,
+                     rank_r: int) -> int:
+    """Disagreement between the INT8 and the FP16 block rankings (Methodology §3,
+    rank-consistency check), as a count of discordant pairs.
+
+    Over the promoted blocks, take the top r = min(rank_r, number promoted) by
+    INT8 block log-mass and the top r by FP16 block log-mass (each ordered by
+    log-mass descending, ties to the lower block index), and form their union U.
+    Every promoted block has both log-masses, so both orders are defined on U;
+    the result is the number of pairs of U that the two orders place the other
+    way round (the Kendall distance of the two rankings restricted to U).  A
+    block that one ranking puts near the top and the other far below it is in
+    U and is discordant with every block it passes, so a large misranking of a
+    heavy block counts many times, while a swap of two neighbours counts once.
+    """
     idx = np.nonzero(promoted)[0]
     if idx.size == 0:
-        return True
+        return 0
     r = min(rank_r, idx.size)
-    return _top_r(ell8[idx], idx, r) == _top_r(ell16[idx], idx, r)
+    U = sorted(set(_top_r(ell8[idx], idx, r)) | set(_top_r(ell16[idx], idx, r)))
+    n = 0
+    for i in range(len(U)):
+        for j in range(i + 1, len(U)):
+            a, b = U[i], U[j]  # a < b: on equal keys the lower index a comes first
+            a_first_8 = ell8[a] >= ell8[b]
+            a_first_16 = ell16[a] >= ell16[b]
+            n += a_first_8 != a_first_16
+    return n
+
+
+def rank_consistent(ell8: np.ndarray, ell16: np.ndarray, promoted: np.ndarray, rank_r: int,
+                    rank_tol: int = 0) -> bool:
+    """Block-ranking consistency check (Methodology §3): the rankings agree when
+    at most rank_tol pairs of the union of the two top-r lists are discordant
+    (rank_discordance).  The pages name the check, not its form; this is the
+    reading used here, calibrated on the synthetic workloads so that single
+    swaps of blocks whose masses INT8 noise cannot separate pass while a
+    shuffled group of near-tied heavy blocks fails (parity unpinned beyond this
+    stated rule).  rank_tol = 0 is the strict reading: the ordered top-r lists
+    must be equal."""
+    return rank_discordance(ell8, ell16, promoted, rank_r) <= rank_tol
 
 
 def decode_group(q16: np.ndarray, u: dict, th: Thresholds) -> dict:
@@ -345,7 +376,7 @@ def decode_group(q16: np.ndarray, u: dict, th: Thresholds) -> dict:
     rank_fail = np.zeros(G, bool)
     if not th.naive:
         for h in range(G):
-            rank_fail[h] = not rank_consistent(ell8[h], ell16[h], P, th.rank_r)
+            rank_fail[h] = not rank_consistent(ell8[h], ell16[h], P, th.rank_r, th.rank_tol)
 
     r_v = float(np.max(u["vmax"].astype(np.float64) - u["vmin"].astype(np.float64))) if T else 0.0
     return dict(out=out, e_key=e_key, e_val=e_val, key_fail=key_fail, rank_fail=rank_fail,

@@ -154,7 +154,7 @@ def default_thresholds(w: Workload) -> dict:
     """Runtime thresholds for a workload.  Only tau_cov and v_tol are named by the
     method; the others are this implementation's choices (all are plain inputs)."""
     th = dict(tau_cov=0.995, eps_key=5e-3, eps_val=float("inf"), v_tol=0.05,
-              rank_r=4, max_expand=4, layer_dense_frac=0.5)
+              rank_r=8, rank_tol=2, max_expand=4, layer_dense_frac=0.5)
     if w.value_dist == "student_t3":
         th["v_tol"] = 5e-3
     return th

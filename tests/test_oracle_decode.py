@@ -150,6 +150,55 @@ def test_rank_rule_on_constructed_orders():
     assert rank_consistent(ell16, ell16[::-1].copy(), np.zeros(6, bool), 4)
 
 
+def test_rank_discordance_hand_cases():
+    """Discordant pairs over the union of the two top-r lists, by hand."""
+    from oracle import rank_discordance
+    ell16 = np.array([5.0, 4.0, 3.0, 2.0, 1.0, 0.0])
+    allp = np.ones(6, bool)
+    # one neighbour swap: U = {0, 1, 2}, one discordant pair
+    assert rank_discordance(np.array([4.0, 5.0, 3.0, 2.0, 1.0, 0.0]), ell16, allp, 3) == 1
+    # the heaviest FP16 block ranked fifth by INT8: U = {0, 1, 2, 3} and block 0
+    # is discordant with each of the three blocks INT8 put above it
+    heavy16 = np.array([10.0, 4.0, 3.0, 2.0, 1.0, 0.0])
+    assert rank_discordance(np.array([0.5, 4.0, 3.0, 2.0, 1.0, 0.0]), heavy16, allp, 3) == 3
+    # a fully reversed top 3 of an otherwise agreeing ranking: 3 pairs
+    assert rank_discordance(np.array([3.0, 4.0, 5.0, 2.0, 1.0, 0.0]), ell16, allp, 3) == 3
+    # equal keys order by the lower index on both sides: no discordance
+    assert rank_discordance(np.array([5.0, 5.0, 3.0, 2.0, 1.0, 0.0]),
+                            np.array([4.0, 4.0, 3.0, 2.0, 1.0, 0.0]), allp, 4) == 0
+    # unpromoted blocks take no part
+    p = allp.copy()
+    p[0] = False
+    assert rank_discordance(np.array([0.5, 4.0, 3.0, 2.0, 1.0, 0.0]), heavy16, p, 3) == 0
+
+
+def test_rank_discordance_brute_force(rng):
+    """Against an independent formulation: each block's position in the full
+    stable order of each ranking, and the pairs of the union whose positions
+    compare differently; rank_tol = 0 is equality of the ordered top-r lists."""
+    from oracle import rank_consistent, rank_discordance
+    for trial in range(400):
+        n = int(rng.integers(1, 14))
+        e16 = np.round(rng.normal(0, 1, n), 1)  # rounding makes ties common
+        e8 = np.round(e16 + rng.normal(0, 0.3, n), 1)
+        P = rng.random(n) < 0.7
+        r = int(rng.integers(0, 6))
+        idx = np.nonzero(P)[0]
+        if idx.size == 0:
+            assert rank_discordance(e8, e16, P, r) == 0
+            continue
+        def positions(key):
+            order = sorted(idx.tolist(), key=lambda j: (-key[j], j))
+            return {j: k for k, j in enumerate(order)}, order
+        p8, o8 = positions(e8)
+        p16, o16 = positions(e16)
+        rr = min(r, idx.size)
+        U = set(o8[:rr]) | set(o16[:rr])
+        want = sum(1 for a in U for b in U if a < b and (p8[a] < p8[b]) != (p16[a] < p16[b]))
+        assert rank_discordance(e8, e16, P, r) == want
+        assert rank_consistent(e8, e16, P, r, 0) == (o8[:rr] == o16[:rr])
+
+
 def test_naive_mode_promotes_nothing(rng):
     q = rng.standard_normal((8, 64)).astype(np.float16)
     units = _units(rng, 2, 6 * BLOCK + 1, 64)
