@@ -202,7 +202,8 @@ def decision_census(cache, qs, th, w, device) -> dict:
     L, B, Hkv, G = w.n_layers, w.batch, w.n_kv_heads, w.group
     c = dict(blocks=0, key_promoted=0, value_promoted=0, heads=0, rungs=[0] * 5, units=0,
              dense_units=0, dense_unit_blocks=0, dense_unit_nonpromoted=0,
-             vp_or_dense_blocks=0, int4_blocks=0, blocks_per_layer=0)
+             vp_or_dense_blocks=0, int4_blocks=0, blocks_per_layer=0, rank_fail=0, key_fail=0)
+    e_key, e_val = [], []
     for layer in range(L):
         tr = cache.alloc_trace(layer)
         o = cache.alloc_outputs()
@@ -231,6 +232,16 @@ def decision_census(cache, qs, th, w, device) -> dict:
         c["heads"] += int(rg.size)
         for r in range(5):
             c["rungs"][r] += int((rg == r).sum())
+        hf = tr["head_flags"].cpu().numpy()
+        c["rank_fail"] += int(((hf & 8) != 0).sum())
+        c["key_fail"] += int(((hf & 4) != 0).sum())
+        cert = rg < 3  # dense heads report 0 for both bounds
+        e_key.append(o[1].cpu().numpy()[cert])
+        e_val.append(o[2].cpu().numpy()[cert])
+    ek, ev = np.concatenate(e_key), np.concatenate(e_val)
+    pct = (50, 90, 99, 100)
+    c["e_key_pct"] = {f"p{q}": float(np.percentile(ek, q)) for q in pct} if ek.size else None
+    c["e_val_pct"] = {f"p{q}": float(np.percentile(ev, q)) for q in pct} if ev.size else None
     return c
 
 
@@ -617,6 +628,11 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "staged_layer_frac": staged,
             "prefetch_copy_gbs": phases.get("prefetch", {}).get("achieved_gbs"),
             "rung_histogram": census["rungs"],
+            "rank_fail_heads": census["rank_fail"],
+            "key_fail_heads": census["key_fail"],
+            "heads": census["heads"],
+            "e_key_percentiles": census["e_key_pct"],
+            "e_val_percentiles": census["e_val_pct"],
         },
         "accuracy": accuracy,
         "phases": phases,
@@ -631,6 +647,96 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     return res
 
 
+# ------------------------------------------------ the larger workloads ----
+
+EXTRA_WORKLOADS = ("llama8b_64k_b4_t3values", "llama8b_128k_needle")
+
+
+def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int = 10,
+                       warmup: int = 3) -> dict:
+    """A few timed steps of a larger workload on one GPU: certified steps/s, the
+    INT8/INT4 path's effective KV GB/s and the streaming kernel's per-launch
+    roofline (CUDA events on the launch stream, in a second, profiled pass)."""
+    import certified_quantized_kv_int8_b200 as cqa
+    w = sk.WORKLOADS[name]
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    th_naive = dataclasses.replace(th, naive=True)
+    L, B, Hq, Hkv, d = w.n_layers, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+    t_setup = time.perf_counter()
+    cache = cqa.Cache(L, B, Hq, Hkv, d, w.ctx, device=device.index)
+    for layer in range(L):
+        K, V = sk.kv_layer(w, layer, 0, w.ctx, device=device)
+        cache.append(layer, K, V)
+        del K, V
+    torch.cuda.synchronize(device)
+    t_setup = time.perf_counter() - t_setup
+    n_q = warmup + cert_steps + 2 * naive_steps + 1
+    qs = [[sk.queries(w, layer, s, device) for layer in range(L)] for s in range(n_q)]
+    outs = cache.alloc_outputs()
+    stream = torch.cuda.current_stream(device)
+
+    def run(first, n, thr):
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for s in range(first, first + n):
+            for layer in range(L):
+                cache.decode(layer, qs[s][layer], thr, outputs=outs, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b) * 1e-3
+
+    for s in range(warmup):
+        run(s, 1, th)
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    t_cert = run(warmup, cert_steps, th)
+    first = warmup + cert_steps
+    run(first, 1, th_naive)  # the INT8/INT4 path's own warm-up
+    t_naive = run(first, naive_steps, th_naive)
+    clk = clocks.stop()
+    cache.profile_begin(1 << 20)
+    run(first + naive_steps, naive_steps, th_naive)
+    nms, nn, _ = cache.profile_end()
+    census = decision_census(cache, qs[warmup + cert_steps - 1], th, w, device)
+    blk_units = sum(n // BLOCK for layer in range(L) for n in cache.row_lengths(layer))
+    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d)
+    peaks = measured_peaks()
+    kv_gbs = t1_bytes * naive_steps / t_naive / 1e9
+    avg = nms["naive"] / nn["naive"]
+    per_launch = t1_bytes / L
+    rec = traffic_record("naive")
+    cache.close()
+    return {
+        "config": {"workload": name, "layers": L, "batch": B, "ctx": w.ctx, "q_heads": Hq,
+                   "kv_heads": Hkv, "head_dim": d},
+        "certified_steps_per_s": cert_steps / t_cert, "certified_steps": cert_steps,
+        "int8_int4_path": {
+            "steps_per_s": naive_steps / t_naive, "steps": naive_steps,
+            "effective_kv_gbs": kv_gbs, "frac_of_hbm_peak": kv_gbs / peaks["hbm_gbs"],
+            "tier1_bytes_per_step": t1_bytes,
+            "roofline": {
+                "kernel": "naive", "bound": "hbm", "achieved": per_launch / (avg * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": per_launch / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "peak_source": f"MEASURED_PEAKS.json hbm_gbs, of {peaks['source']}",
+                "avg_launch_ms": avg, "algorithmic_bytes_per_launch": per_launch,
+                "traffic": (rec["dram_bytes_per_block"] * blk_units * Hkv / L if rec else None),
+            },
+        },
+        "promotion": {
+            "key_promoted_frac": census["key_promoted"] / max(1, census["blocks"]),
+            "value_promoted_frac": census["value_promoted"] / max(1, census["blocks"]),
+            "dense_unit_frac": census["dense_units"] / max(1, census["units"]),
+            "rung_histogram": census["rungs"], "rank_fail_heads": census["rank_fail"],
+            "heads": census["heads"],
+            "e_key_percentiles": census["e_key_pct"], "e_val_percentiles": census["e_val_pct"],
+        },
+        "clocks": clk,
+        "setup_s": t_setup,
+    }
+
+
 # --------------------------------------------------------- oracle timing ----
 
 def oracle_sample_seconds(w: sk.Workload, layer: int, b: int, th) -> tuple[float, dict]:
@@ -642,7 +748,7 @@ def oracle_sample_seconds(w: sk.Workload, layer: int, b: int, th) -> tuple[float
     q = sk.queries(w, layer, 0, "cpu")[b].numpy()
     d = th.float32_rounded()
     oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
-             rank_r=d["rank_r"], max_expand=d["max_expand"],
+             rank_r=d["rank_r"], rank_tol=d["rank_tol"], max_expand=d["max_expand"],
              layer_dense_frac=d["layer_dense_frac"])
     t0 = time.perf_counter()
     decode(q, units, oth)
@@ -707,7 +813,7 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
     units = [build_unit(K[g].numpy(), V[g].numpy()) for g in range(w.n_kv_heads)]
     d = th.float32_rounded()
     oth = OT(tau_cov=d["tau_cov"], eps_key=d["eps_key"], eps_val=d["eps_val"], v_tol=d["v_tol"],
-             rank_r=d["rank_r"], max_expand=d["max_expand"],
+             rank_r=d["rank_r"], rank_tol=d["rank_tol"], max_expand=d["max_expand"],
              layer_dense_frac=d["layer_dense_frac"])
     qs = [sk.queries(w, 0, s, "cpu")[0].numpy() for s in range(args.warmup + args.steps)]
     for s in range(args.warmup):
@@ -754,6 +860,9 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only the first N layers (profiling captures; the reported "
                          "line then covers N layers, not the workload's step)")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the few timed steps of the 64K x B4 and 128K workloads that the "
+                         "default single-GPU line adds under `workloads`")
     ap.add_argument("--clocks-csv", default=None,
                     help="keep the nvidia-smi samples of the timed region in this file")
     args = ap.parse_args(argv)
@@ -779,6 +888,11 @@ def main(argv=None):
         build()  # no-op once rank 0 built it
     device = torch.device("cuda", local)
     res = run_ours(args, w, ws, rank, dist, device)
+    if (res is not None and ws == 1 and args.layers is None and not args.no_extra_workloads
+            and w.name == DEFAULT_WORKLOAD):
+        # the larger single-GPU workloads, a few steps each (one GPU only: the
+        # 64K x B4 workload holds 32 GiB of pinned host memory)
+        res["workloads"] = {n: run_extra_workload(n, device) for n in EXTRA_WORKLOADS}
     if rank == 0 and res is not None:
         if ws == 1 and not args.no_cpu_baseline:
             import certified_quantized_kv_int8_b200 as cqa

@@ -43,6 +43,7 @@ EXPORTED_SYMBOLS = (
     "cqa_quantize_append", "cqa_quantize_append_row", "cqa_decode", "cqa_dense_reference", "cqa_debug_export", "cqa_error_string",
     "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
     "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait",
+    "cqa_test_inject_fault",
 )
 
 PHASES = ("append_seal", "append_tail", "score", "select", "promote", "decide", "dense_keys",
@@ -136,13 +137,15 @@ def load_library() -> ctypes.CDLL:
     lib.cqa_set_key_prefetch.argtypes = [vp, i32, ctypes.c_float]
     lib.cqa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     lib.cqa_selftest_bounded_wait.argtypes = [vp, ctypes.c_int32]
+    lib.cqa_test_inject_fault.argtypes = [i32, i32]
     lib.cqa_error_string.argtypes = [i32]
     lib.cqa_error_string.restype = ctypes.c_char_p
     for name in ("cqa_cache_create", "cqa_cache_destroy", "cqa_cache_length",
                  "cqa_cache_row_lengths", "cqa_quantize_append", "cqa_quantize_append_row",
                  "cqa_decode", "cqa_dense_reference",
                  "cqa_profile_begin", "cqa_profile_end", "cqa_dense_attention_noalloc",
-                 "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait"):
+                 "cqa_set_key_prefetch", "cqa_device_status", "cqa_selftest_bounded_wait",
+                 "cqa_test_inject_fault"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -268,6 +271,14 @@ def cqa_selftest_bounded_wait(handle, polls: int = 1000):
     """Launch a kernel whose bounded wait must give up (see include/cqa.h)."""
     return _check(load_library().cqa_selftest_bounded_wait(handle, int(polls)),
                   "cqa_selftest_bounded_wait")
+
+
+FAULT_NONE, FAULT_PINNED_ALLOC, FAULT_PREFETCH_COPY = 0, 1, 2
+
+
+def cqa_test_inject_fault(site: int, skip: int = 0):
+    """Arm the library's host-side fault injection (a test hook, see cqa.h)."""
+    _check(load_library().cqa_test_inject_fault(int(site), int(skip)), "cqa_test_inject_fault")
 
 
 def cqa_dense_attention_noalloc(q, k, v, out, stream=None):

@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <new>
@@ -70,6 +71,27 @@ struct cqa_cache {
 };
 
 namespace {
+
+// Host-side fault injection (cqa_test_inject_fault): the armed site fails once,
+// after `skip` calls of it have passed.  Off unless a caller arms it.
+std::atomic<int> g_fault_site{CQA_FAULT_NONE};
+std::atomic<int> g_fault_skip{0};
+
+bool fault_hit(int site) {
+  if (g_fault_site.load() != site) return false;
+  if (g_fault_skip.fetch_sub(1) > 0) return false;
+  g_fault_site.store(CQA_FAULT_NONE);
+  return true;
+}
+
+// cudaHostAlloc, or the injected failure of a pinned allocation
+cudaError_t pinned_alloc(void** p, size_t bytes, unsigned flags) {
+  if (fault_hit(CQA_FAULT_PINNED_ALLOC)) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaHostAlloc(p, bytes, flags);
+}
 
 struct DeviceGuard {
   int prev = -1;
@@ -227,7 +249,8 @@ int staged_slot(const cqa_cache* c, int layer) {
 // copy stream, after all work already queued on `s` (the appends that wrote
 // them) and after the slot's last reader.  Each batch row copies its own
 // sealed blocks (one copy for all rows when their block counts agree).
-// Returns the slot or -1.
+// Returns the slot, -1 when there is nothing to copy, or -2 when a CUDA call
+// failed (the slot is then marked empty).
 int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
   const int nb = max_len(c, layer) / BLK;
   if (nb == 0) return -1;
@@ -242,11 +265,12 @@ int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
   const int32_t* L = row_lens(c, layer);
   bool same = true;
   for (int b = 1; b < B; ++b) same = same && (L[b] / BLK == L[0] / BLK);
-  if (cudaEventRecord(c->ev_main, s) != cudaSuccess) return -1;
-  if (cudaStreamWaitEvent(c->side, c->ev_main, 0) != cudaSuccess) return -1;
-  if (cudaStreamWaitEvent(c->side, c->ev_free[slot], 0) != cudaSuccess) return -1;
+  if (cudaEventRecord(c->ev_main, s) != cudaSuccess) return -2;
+  if (cudaStreamWaitEvent(c->side, c->ev_main, 0) != cudaSuccess) return -2;
+  if (cudaStreamWaitEvent(c->side, c->ev_free[slot], 0) != cudaSuccess) return -2;
   const int timed = c->prof_on ? 1 : 0;
   cudaError_t e = run_phase(c, CQA_PHASE_PREFETCH, c->side, timed, [&] {
+    if (fault_hit(CQA_FAULT_PREFETCH_COPY)) return cudaErrorInvalidValue;
     if (same)
       return cudaMemcpy2DAsync(c->kstage[slot], pitch, src, pitch, (size_t)nb * blk_bytes, units,
                                cudaMemcpyHostToDevice, c->side);
@@ -263,7 +287,7 @@ int issue_prefetch(cqa_cache* c, int layer, int avoid_slot, cudaStream_t s) {
   });
   if (e != cudaSuccess || cudaEventRecord(c->ev_ready[slot], c->side) != cudaSuccess) {
     c->stage_layer[slot] = -1;
-    return -1;
+    return -2;
   }
   c->stage_layer[slot] = layer;
   c->stage_nb[slot] = nb;
@@ -412,9 +436,9 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   }
 
   cc->tier2_bytes = units * st.tier2 * 2;
-  if (cudaHostAlloc(&cc->k2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
+  if (pinned_alloc(&cc->k2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
           cudaSuccess ||
-      cudaHostAlloc(&cc->v2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
+      pinned_alloc(&cc->v2_host, cc->tier2_bytes, cudaHostAllocMapped | cudaHostAllocPortable) !=
           cudaSuccess) {
     cudaGetLastError();
     cqa_cache_destroy(cc);
@@ -457,8 +481,8 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
     cqa_cache_destroy(cc);
     return CQA_ERR_CUDA;
   }
-  if (cudaHostAlloc((void**)&cc->promo_host, units * sizeof(int32_t),
-                    cudaHostAllocMapped | cudaHostAllocPortable) != cudaSuccess) {
+  if (pinned_alloc((void**)&cc->promo_host, units * sizeof(int32_t),
+                   cudaHostAllocMapped | cudaHostAllocPortable) != cudaSuccess) {
     cudaGetLastError();
     cqa_cache_destroy(cc);
     return CQA_ERR_OOM;
@@ -628,15 +652,19 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   const bool naive = tv.naive != 0;
   const bool post_check = !naive && !isinf(tv.eps_val);
   // keys of this layer staged by an earlier call, or staged now; then the next layer's
+  // (a failed copy call is reported before any kernel is launched, so the
+  // caller's outputs are left untouched)
   int slot = -1;
   if (!naive) {
     slot = staged_slot(cc, layer);
     if (slot < 0 && want_prefetch(cc, layer)) slot = issue_prefetch(cc, layer, -1, s);
+    if (slot == -2) return CQA_ERR_CUDA;
     // the next layer's keys, copied while this layer runs: the copy shares the
     // host link with this layer's value pass, which keeps the link busy through
     // the scoring and selection phases that do not use it
     const int next = (layer + 1) % cc->cfg.n_layers;
-    if (next != layer && want_prefetch(cc, next)) issue_prefetch(cc, next, slot, s);
+    if (next != layer && want_prefetch(cc, next) && issue_prefetch(cc, next, slot, s) == -2)
+      return CQA_ERR_CUDA;
   }
   const __half* kstage = slot >= 0 ? cc->kstage[slot] : nullptr;
   const int stage_nb = slot >= 0 ? cc->stage_nb[slot] : 0;
@@ -805,6 +833,15 @@ int cqa_selftest_bounded_wait(cqa_cache* cc, int32_t polls) {
   if (!dg.ok) return CQA_ERR_CUDA;
   bounded_wait_selftest_kernel<<<1, 32>>>(cc->sc.err, (uint32_t)polls);
   return cudaGetLastError() == cudaSuccess ? CQA_OK : CQA_ERR_CUDA;
+}
+
+int cqa_test_inject_fault(int site, int skip) {
+  if (site < CQA_FAULT_NONE || site > CQA_FAULT_PREFETCH_COPY || skip < 0)
+    return CQA_ERR_INVALID_ARG;
+  g_fault_site.store(CQA_FAULT_NONE);
+  g_fault_skip.store(skip);
+  g_fault_site.store(site);
+  return CQA_OK;
 }
 
 int cqa_set_key_prefetch(cqa_cache* cc, int mode, float min_fraction) {

@@ -3,12 +3,16 @@
 // file-scope device array.
 //
 // Who needs this: callers that cannot call cudaMalloc.  Typical cases are
-// code that runs while a stream is being captured into a CUDA graph (an
-// allocation there either fails or breaks the capture), hosts that hand a
-// fixed memory budget to several libraries and own the only allocator, and
-// latency-critical paths where cudaMalloc/cudaFree may synchronise the
-// device.  Such callers still pass their own inputs and outputs; the only
-// memory this entry point needs beyond them is the scratch array below.
+// hosts that hand a fixed memory budget to several libraries and own the only
+// device allocator (memory a library allocated on its own would be memory the
+// host already promised elsewhere), and latency-critical paths where
+// cudaMalloc/cudaFree may synchronise the device.  Such callers still pass
+// their own inputs and outputs; the only memory this entry point needs beyond
+// them is the scratch array below.
+//
+// Shapes: head_dim 64 or 128, n_q_heads / n_kv_heads in {1, 2, 4, 8} (8 only
+// at head_dim 128), batch * n_kv_heads <= 65535, and the partials of one
+// chunk per kv head within the array's 4 MiB.
 //
 // The paper has no counterpart of this entry point; it is a deployment
 // convenience of this library.

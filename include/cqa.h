@@ -219,6 +219,24 @@ int cqa_device_status(cqa_cache* cache, int32_t* status);
  * nothing faults or hangs.  Runs on the legacy default stream. */
 int cqa_selftest_bounded_wait(cqa_cache* cache, int32_t polls);
 
+/* Host-side fault injection, a test hook for the library's error paths
+ * (Key Contributions: recovery must be deterministic, so its failure paths are
+ * exercised without faulting a GPU).  Off unless armed; process-wide.  The
+ * armed site fails once, on the host and without calling CUDA for it, after
+ * `skip` of its calls have passed, and then disarms:
+ *   CQA_FAULT_PINNED_ALLOC  a pinned host allocation of cqa_cache_create (there
+ *                           are three: Tier-2 keys, Tier-2 values, the promotion
+ *                           counters); the create returns CQA_ERR_OOM after
+ *                           freeing everything it had allocated;
+ *   CQA_FAULT_PREFETCH_COPY a copy of the whole-layer key prefetch; cqa_decode
+ *                           returns CQA_ERR_CUDA before launching any kernel, so
+ *                           its outputs are left untouched, and the slot is
+ *                           marked empty.
+ * CQA_FAULT_NONE disarms.  CQA_ERR_INVALID_ARG for an unknown site or skip < 0.
+ * Arming is not synchronised with calls made by other threads. */
+enum { CQA_FAULT_NONE = 0, CQA_FAULT_PINNED_ALLOC = 1, CQA_FAULT_PREFETCH_COPY = 2 };
+int cqa_test_inject_fault(int site, int skip);
+
 /* Whole-layer key prefetch.  Promotion reads the FP16 keys of the selected
  * blocks from Tier 2.  When a layer's last decode promoted nearly all of its
  * blocks, copying the layer's sealed keys to device memory with the copy
@@ -272,16 +290,19 @@ int cqa_profile_end(cqa_cache* cache, double* ms, int64_t* launches);
 
 /* Exact attention softmax(q K^T / sqrt(head_dim)) V over FP16 keys and values
  * that the caller holds in device memory, computed without allocating any
- * memory.  The paper has no counterpart of this entry point: it exists for
- * callers that cannot call cudaMalloc, e.g. code running while a stream is
- * captured into a CUDA graph (an allocation there fails or breaks the
- * capture), hosts whose single allocator is owned by another framework under
- * a fixed memory budget, and latency-critical paths where cudaMalloc/cudaFree
- * may synchronise the device.
+ * memory.  The paper has no counterpart of this entry point.  It exists for
+ * callers that cannot call cudaMalloc: hosts whose single device allocator is
+ * owned by another framework under a fixed memory budget (a library that
+ * allocates on its own there takes memory the host has already promised
+ * elsewhere), and latency-critical paths where cudaMalloc/cudaFree may
+ * synchronise the device and stall every stream.
  *
  * q_fp16: device fp16 [batch][n_q_heads][head_dim]; k_fp16, v_fp16: device
  * fp16 [batch][n_kv_heads][n_tokens][head_dim]; out: device fp32
  * [batch][n_q_heads][head_dim]; all 16-byte aligned, owned by the caller.
+ * Supported shapes: head_dim 64 or 128; n_q_heads / n_kv_heads (an integer)
+ * in {1, 2, 4, 8}, except 8 at head_dim 64; batch, heads and n_tokens >= 1;
+ * batch * n_kv_heads <= 65535.  Other shapes return CQA_ERR_INVALID_ARG.
  * The split-K partials live in a file-scope device array of
  * CQA_NOALLOC_SCRATCH_BYTES; shapes whose partials cannot fit (batch *
  * n_kv_heads * (n_q_heads / n_kv_heads) * (head_dim + 3) * 4 bytes above it)
