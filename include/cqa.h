@@ -113,10 +113,14 @@ typedef struct cqa_trace {
   float* ell_res;       /* [batch][n_q_heads] log-mass of the exact residual block (-inf if empty) */
 } cqa_trace;
 
-/* Allocate both tiers for `cfg` on cfg->device: Tier 1 and scratch in device
- * memory, Tier 2 (n_layers * batch * n_kv_heads * max_ctx * head_dim * 2 fp16)
- * in pinned, device-mapped host memory, and the two key-staging buffers of
- * cqa_set_key_prefetch.  *out receives the handle. */
+/* Allocate both tiers for `cfg` on cfg->device (Methodology §1, tiered
+ * storage: Tier 1 holds the compressed cache in device memory, Tier 2 the FP16
+ * originals in pinned system RAM): Tier 1 and scratch in device memory, Tier 2
+ * (n_layers * batch * n_kv_heads * max_ctx * head_dim * 2 fp16) in pinned,
+ * device-mapped host memory, and the two key-staging buffers of
+ * cqa_set_key_prefetch.  *out receives the handle.  CQA_ERR_INVALID_ARG for an
+ * unsupported shape, CQA_ERR_OOM when a device or pinned allocation fails
+ * (everything allocated so far is freed and *out stays NULL). */
 int cqa_cache_create(const cqa_config* cfg, cqa_cache** out);
 
 /* Free everything the cache owns (synchronises the device first).  NULL is a no-op. */
@@ -172,7 +176,8 @@ int cqa_decode(cqa_cache* cache, int layer, const void* q_fp16, const cqa_thresh
 
 /* Exact attention softmax(q K^T / sqrt(head_dim)) V of `layer` over the FP16
  * originals (Tier 2 plus the residual block), fp32 accumulation: the O_dense
- * the fallback ladder returns.  q_fp16 and out as in cqa_decode, each row
+ * that deterministic recovery returns (Key Contributions; Methodology §1,
+ * fallback mechanism) and the dense rungs 3-4 of the ladder compute.  q_fp16 and out as in cqa_decode, each row
  * over its own tokens; CQA_ERR_EMPTY if some row holds no token. */
 int cqa_dense_reference(cqa_cache* cache, int layer, const void* q_fp16, float* out, void* stream);
 

@@ -10,6 +10,7 @@ shares no code, table or constant with the CUDA sources.
 from .cqa_oracle import (  # noqa: F401
     BLOCK,
     VGROUP,
+    fp16_round_up,
     quantize_keys_block,
     quantize_values_block,
     pack_int4,

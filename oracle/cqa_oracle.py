@@ -45,18 +45,35 @@ F32 = np.float32
 # Tier 1 encoding (Methodology §1)
 # ---------------------------------------------------------------------------
 
-def quantize_keys_block(k16: np.ndarray):
+def fp16_round_up(x: np.ndarray) -> np.ndarray:
+    """The smallest IEEE binary16 value >= x, for float32 0 <= x <= 65504, returned
+    as float32: round to nearest, then one step up when that fell below x."""
+    h = np.asarray(x, F32).astype(np.float16)
+    low = h.astype(F32) < x
+    h[low] = np.nextafter(h[low], np.float16(np.inf))
+    return h.astype(F32)
+
+
+def quantize_keys_block(k16: np.ndarray, fp16_meta: bool = False):
     """Per-channel symmetric INT8 keys for one block (Methodology §1).
 
-    Reading: one float32 scale per (block, channel) over the block's tokens,
-    s = amax / 127, code = clamp(round_half_even(k / s), -127, 127); an
-    all-zero channel gets s = 0 and codes 0.  Dequantised key = code * s.
+    Reading: one scale per (block, channel) over the block's tokens,
+    s = amax / 127 (float32), code = clamp(round_half_even(k / s), -127, 127);
+    an all-zero channel gets s = 0 and codes 0.  Dequantised key = code * s.
+
+    fp16_meta: the scale is stored as binary16, rounded up (the smallest fp16
+    >= amax / 127), and the codes are taken against that stored scale.  Then
+    |k / s| <= 127 still (no code is clamped) and |k - code * s| <= s / 2 for
+    the stored s, so Delta computed from the stored scales stays a valid
+    per-token perturbation bound.
 
     k16: float16 [BLOCK, d].  Returns (codes int8 [BLOCK, d], scale float32 [d]).
     """
     k = k16.astype(F32)
     amax = np.max(np.abs(k), axis=0)
     scale = (amax / F32(127.0)).astype(F32)
+    if fp16_meta:
+        scale = fp16_round_up(scale)
     ratio = np.zeros_like(k)
     nz = scale > 0
     ratio[:, nz] = k[:, nz] / scale[nz]
@@ -64,7 +81,7 @@ def quantize_keys_block(k16: np.ndarray):
     return codes, scale
 
 
-def quantize_values_block(v16: np.ndarray):
+def quantize_values_block(v16: np.ndarray, fp16_meta: bool = False):
     """Per-group asymmetric INT4 values for one block, with its error annotation.
 
     Reading (Methodology §1, "per-group INT4 values ... scales/offsets ...
@@ -75,6 +92,12 @@ def quantize_values_block(v16: np.ndarray):
     operation; eta_b = max over the block of |v - v_hat| (float32), the
     measured reconstruction error written when the originals are at hand.
 
+    fp16_meta: offset and scale are stored as binary16.  The offset, the min of
+    binary16 values, is one of them and stays exact; the scale is rounded up
+    (the smallest fp16 >= (max - min) / 15), so (v - z) / s <= 15 and no code is
+    clamped; v_hat and eta_b use the stored values, so eta_b still bounds
+    |v - v_hat| exactly as measured.
+
     v16: float16 [BLOCK, d].  Returns (codes uint8 [BLOCK, d] unpacked,
     scale float32 [BLOCK, d/VGROUP], offset float32 [BLOCK, d/VGROUP],
     v_hat float32 [BLOCK, d], eta float32 scalar).
@@ -84,6 +107,8 @@ def quantize_values_block(v16: np.ndarray):
     lo = v.min(axis=2)
     hi = v.max(axis=2)
     scale = ((hi - lo).astype(F32) / F32(15.0)).astype(F32)
+    if fp16_meta:
+        scale = fp16_round_up(scale)
     diff = (v - lo[:, :, None]).astype(F32)
     ratio = np.zeros_like(v)
     nz = scale > 0
@@ -107,14 +132,15 @@ def unpack_int4(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def build_unit(K16: np.ndarray, V16: np.ndarray) -> dict:
+def build_unit(K16: np.ndarray, V16: np.ndarray, fp16_meta: bool = False) -> dict:
     """Tier-1 and Tier-2 contents of one (layer, batch row, kv head) after T tokens.
 
     Sealed blocks are the nb = T // BLOCK complete blocks; the r = T % BLOCK
     newest tokens form the residual block, kept exact in FP16 (Delta = 0,
     eta = 0).  Each sealed block depends only on its own tokens, so the result
     is independent of how the tokens were appended.  vmin / vmax are the
-    per-channel value ranges over all T tokens.
+    per-channel value ranges over all T tokens.  fp16_meta: scales and offsets
+    stored as binary16 (quantize_keys_block, quantize_values_block).
     """
     T, d = K16.shape
     nb = T // BLOCK
@@ -127,8 +153,8 @@ def build_unit(K16: np.ndarray, V16: np.ndarray) -> dict:
     eta = np.zeros(nb, F32)
     for j in range(nb):
         sl = slice(j * BLOCK, (j + 1) * BLOCK)
-        kc[j], ks[j] = quantize_keys_block(K16[sl])
-        vc[j], vs[j], vz[j], vh[j], eta[j] = quantize_values_block(V16[sl])
+        kc[j], ks[j] = quantize_keys_block(K16[sl], fp16_meta)
+        vc[j], vs[j], vz[j], vh[j], eta[j] = quantize_values_block(V16[sl], fp16_meta)
     Vf = V16.astype(F32)
     vmin = Vf.min(axis=0) if T else np.zeros(d, F32)
     vmax = Vf.max(axis=0) if T else np.zeros(d, F32)

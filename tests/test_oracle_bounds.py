@@ -81,21 +81,22 @@ def test_brute_force_extreme_perturbations(rng):
     assert worst_ratio > 0.3  # the bound is not vacuous on these cases
 
 
-def _unit_from(rng, T, d, outlier=10.0, heavy_v=False):
+def _unit_from(rng, T, d, outlier=10.0, heavy_v=False, fp16_meta=False):
     K = rng.standard_normal((T, d))
     K[:, :4] *= outlier
     V = rng.standard_t(3, (T, d)) if heavy_v else rng.standard_normal((T, d))
-    return build_unit(K.astype(np.float16), V.astype(np.float16))
+    return build_unit(K.astype(np.float16), V.astype(np.float16), fp16_meta)
 
 
 @pytest.mark.parametrize("tau", [0.5, 0.9, 0.995])
 @pytest.mark.parametrize("heavy_v", [False, True])
-def test_bounds_hold_on_decoded_heads(rng, tau, heavy_v):
+@pytest.mark.parametrize("fp16_meta", [False, True])
+def test_bounds_hold_on_decoded_heads(rng, tau, heavy_v, fp16_meta):
     d, G, Hkv = 64, 2, 2
     for trial in range(3):
         T = int(rng.integers(4, 20)) * BLOCK + int(rng.integers(0, BLOCK))
         units = [_unit_from(rng, T, d, outlier=float(rng.choice([1.0, 10.0, 40.0])),
-                            heavy_v=heavy_v) for _ in range(Hkv)]
+                            heavy_v=heavy_v, fp16_meta=fp16_meta) for _ in range(Hkv)]
         q = rng.standard_normal((G * Hkv, d)).astype(np.float16)
         th = Thresholds(tau_cov=tau, eps_key=1.0, v_tol=float("inf"), rank_r=0,
                         layer_dense_frac=2.0)

@@ -105,3 +105,71 @@ def test_build_unit_blocks_and_residual(rng):
     np.testing.assert_array_equal(u["kscale"][1], s1)
     np.testing.assert_array_equal(u["vmin"], V.astype(np.float32).min(0))
     np.testing.assert_array_equal(u["vmax"], V.astype(np.float32).max(0))
+
+
+# ---- binary16 metadata with directed rounding ----
+
+def _all_finite_fp16_ascending():
+    h = np.arange(1 << 16, dtype=np.uint16).view(np.float16)
+    h = h[np.isfinite(h)].astype(np.float32)
+    return np.unique(h)
+
+
+def test_fp16_round_up_brute_force(rng):
+    """The smallest binary16 >= x, against a search over every finite binary16."""
+    from oracle import fp16_round_up
+    table = _all_finite_fp16_ascending()
+    x = np.concatenate([
+        rng.uniform(0, 1, 2000), rng.uniform(0, 1e-3, 2000) ** 2, rng.uniform(0, 600, 2000),
+        table[(table >= 0) & (table < 600)][::97],  # exact binary16 values map to themselves
+        [0.0, 1.0 / 127, 1.0 / 15, 65504.0],
+    ]).astype(np.float32)
+    got = fp16_round_up(x)
+    want = table[np.searchsorted(table, x, side="left")]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_fp16_meta_hand_fixture():
+    g = load("fp16_meta_hand.txt")
+    d = 32
+    K = np.zeros((BLOCK, d), np.float16)
+    K[:5, 0] = g["k"]
+    codes, scale = quantize_keys_block(K, fp16_meta=True)
+    assert float(scale[0]) == float(g["key_scale"][0])
+    np.testing.assert_array_equal(codes[:5, 0], g["key_codes"].astype(np.int8))
+    V = np.zeros((BLOCK, d), np.float16)
+    V[0, :4] = g["v"]
+    vcodes, vscale, voff, v_hat, eta = quantize_values_block(V, fp16_meta=True)
+    assert float(vscale[0, 0]) == float(g["value_scale"][0])
+    assert float(voff[0, 0]) == 0.0
+    np.testing.assert_array_equal(vcodes[0, :4], g["value_codes"].astype(np.uint8))
+    assert float(eta) == float(g["eta"][0])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("heavy", [False, True])
+def test_fp16_meta_bounds_hold(rng, d, heavy):
+    """With binary16 metadata: the scales are binary16 values rounded up from the
+    float32 ones, no code is clamped, and the errors stay within half a stored
+    step (keys) and within the measured eta_b (values)."""
+    for blk in _blocks(rng, 12, d, heavy):
+        codes32, s32 = quantize_keys_block(blk)
+        codes, s = quantize_keys_block(blk, fp16_meta=True)
+        assert np.all(s.astype(np.float16).astype(np.float32) == s)
+        assert np.all(s >= s32)
+        ratio = np.abs(blk.astype(np.float64)) / np.where(s > 0, s, 1.0)
+        assert np.all(ratio <= 127.0 * (1 + 2.0 ** -22))
+        err = np.abs(blk.astype(np.float64) - codes.astype(np.float64) * s.astype(np.float64))
+        assert np.all(err <= s.astype(np.float64) * (0.5 + 127 * 2.0 ** -23))
+        vc, vs, vz, vh, eta = quantize_values_block(blk, fp16_meta=True)
+        vc32, vs32, vz32, vh32, eta32 = quantize_values_block(blk)
+        assert np.all(vs.astype(np.float16).astype(np.float32) == vs)
+        assert np.all(vz.astype(np.float16).astype(np.float32) == vz)
+        np.testing.assert_array_equal(vz, vz32)  # the offset is the group min, exact
+        assert np.all(vs >= vs32)
+        v = blk.astype(np.float32).reshape(BLOCK, d // VGROUP, VGROUP)
+        r = (v - vz[:, :, None]) / np.where(vs > 0, vs, 1.0)[:, :, None]
+        assert np.all(r <= 15.0 * (1 + 2.0 ** -22))
+        verr = np.abs(blk.astype(np.float32) - vh)
+        assert float(verr.max()) == float(eta)
+        assert float(eta) <= float(vs.max()) * (0.5 + 2.0 ** -20)
