@@ -60,9 +60,11 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def tier1_bytes_per_block(d: int) -> int:
-    """INT8 key codes + key scales + INT4 value codes + value scale/offset + eta_b."""
-    return BLOCK * d + 4 * d + BLOCK * d // 2 + BLOCK * (d // 32) * 8 + 4
+def tier1_bytes_per_block(d: int, meta_fp16: bool = False) -> int:
+    """INT8 key codes + key scales + INT4 value codes + value scale/offset + eta_b
+    (scales and offsets 2 bytes each with binary16 metadata, else 4)."""
+    m = 2 if meta_fp16 else 4
+    return BLOCK * d + m * d + BLOCK * d // 2 + BLOCK * (d // 32) * 2 * m + 4
 
 
 def dist_env():
@@ -313,7 +315,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     max_ctx = w.ctx + (total_steps if appends else 0)
     wr = dataclasses.replace(w, seed=w.seed + rank)  # independent replica per rank
 
-    cache = cqa.Cache(L, B, Hq, Hkv, d, max_ctx, device=device.index)
+    cache = cqa.Cache(L, B, Hq, Hkv, d, max_ctx, device=device.index, meta_fp16=args.meta_fp16)
     lens0 = sk.row_lengths(w)
     for layer in range(L):
         if w.row_ctx:  # a ragged batch: each row appended on its own
@@ -496,7 +498,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         vtol_sweep = rows
     # sealed blocks of all (layer, batch row) units per kv head, lengths at the end
     blk_units = sum(n // BLOCK for layer in range(L) for n in cache.row_lengths(layer))
-    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d)  # per step
+    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d, args.meta_fp16)  # per step
     peaks = measured_peaks()
     kv_gbs = t1_bytes * n_naive / n_max / 1e9 * ws
 
@@ -603,6 +605,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "ctx": w.ctx, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
             **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {}),
             "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
+            "meta_fp16": bool(args.meta_fp16),
             "l2": "inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (
                 t1_bytes / 2 ** 30),
             "thresholds": dataclasses.asdict(th),
@@ -653,7 +656,7 @@ EXTRA_WORKLOADS = ("llama8b_64k_b4_t3values", "llama8b_128k_needle")
 
 
 def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int = 10,
-                       warmup: int = 3) -> dict:
+                       warmup: int = 3, meta_fp16: bool = False) -> dict:
     """A few timed steps of a larger workload on one GPU: certified steps/s, the
     INT8/INT4 path's effective KV GB/s and the streaming kernel's per-launch
     roofline (CUDA events on the launch stream, in a second, profiled pass)."""
@@ -663,7 +666,7 @@ def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int 
     th_naive = dataclasses.replace(th, naive=True)
     L, B, Hq, Hkv, d = w.n_layers, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
     t_setup = time.perf_counter()
-    cache = cqa.Cache(L, B, Hq, Hkv, d, w.ctx, device=device.index)
+    cache = cqa.Cache(L, B, Hq, Hkv, d, w.ctx, device=device.index, meta_fp16=meta_fp16)
     for layer in range(L):
         K, V = sk.kv_layer(w, layer, 0, w.ctx, device=device)
         cache.append(layer, K, V)
@@ -700,7 +703,7 @@ def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int 
     nms, nn, _ = cache.profile_end()
     census = decision_census(cache, qs[warmup + cert_steps - 1], th, w, device)
     blk_units = sum(n // BLOCK for layer in range(L) for n in cache.row_lengths(layer))
-    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d)
+    t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d, meta_fp16)
     peaks = measured_peaks()
     kv_gbs = t1_bytes * naive_steps / t_naive / 1e9
     avg = nms["naive"] / nn["naive"]
@@ -709,7 +712,7 @@ def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int 
     cache.close()
     return {
         "config": {"workload": name, "layers": L, "batch": B, "ctx": w.ctx, "q_heads": Hq,
-                   "kv_heads": Hkv, "head_dim": d},
+                   "kv_heads": Hkv, "head_dim": d, "meta_fp16": meta_fp16},
         "certified_steps_per_s": cert_steps / t_cert, "certified_steps": cert_steps,
         "int8_int4_path": {
             "steps_per_s": naive_steps / t_naive, "steps": naive_steps,
@@ -860,6 +863,9 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only the first N layers (profiling captures; the reported "
                          "line then covers N layers, not the workload's step)")
+    ap.add_argument("--meta-fp16", action="store_true",
+                    help="caches store Tier-1 scales and offsets as binary16 (212 instead of "
+                         "232 bytes per token and kv head)")
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="skip the few timed steps of the 64K x B4 and 128K workloads that the "
                          "default single-GPU line adds under `workloads`")
@@ -892,7 +898,8 @@ def main(argv=None):
             and w.name == DEFAULT_WORKLOAD):
         # the larger single-GPU workloads, a few steps each (one GPU only: the
         # 64K x B4 workload holds 32 GiB of pinned host memory)
-        res["workloads"] = {n: run_extra_workload(n, device) for n in EXTRA_WORKLOADS}
+        res["workloads"] = {n: run_extra_workload(n, device, meta_fp16=args.meta_fp16)
+                            for n in EXTRA_WORKLOADS}
     if rank == 0 and res is not None:
         if ws == 1 and not args.no_cpu_baseline:
             import certified_quantized_kv_int8_b200 as cqa

@@ -55,7 +55,7 @@ class _Config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int32), ("batch", ctypes.c_int32),
                 ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
-                ("device", ctypes.c_int32)]
+                ("device", ctypes.c_int32), ("meta_fp16", ctypes.c_int32)]
 
 
 class _Thresholds(ctypes.Structure):
@@ -177,8 +177,10 @@ def cqa_error_string(code: int) -> str:
     return load_library().cqa_error_string(int(code)).decode()
 
 
-def cqa_cache_create(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0):
-    cfg = _Config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device)
+def cqa_cache_create(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0,
+                     meta_fp16=False):
+    cfg = _Config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device,
+                  1 if meta_fp16 else 0)
     h = ctypes.c_void_p()
     _check(load_library().cqa_cache_create(ctypes.byref(cfg), ctypes.byref(h)), "cqa_cache_create")
     return h
@@ -300,17 +302,21 @@ def cqa_dense_attention_noalloc(q, k, v, out, stream=None):
 class Cache:
     """A cqa_cache handle with its shape; methods mirror the C entry points."""
 
-    def __init__(self, n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0):
+    def __init__(self, n_layers, batch, n_q_heads, n_kv_heads, head_dim, max_ctx, device=0,
+                 meta_fp16=False):
         self.n_layers, self.batch = n_layers, batch
         self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
-        self.max_ctx, self.device = max_ctx, device
+        self.max_ctx, self.device, self.meta_fp16 = max_ctx, device, bool(meta_fp16)
         self.handle = cqa_cache_create(n_layers, batch, n_q_heads, n_kv_heads, head_dim,
-                                       max_ctx, device)
+                                       max_ctx, device, meta_fp16)
 
     def close(self):
-        if self.handle is not None and self.handle.value:
-            cqa_cache_destroy(self.handle)
-        self.handle = None
+        # cqa_cache_destroy frees everything even when it reports an error (a
+        # failed device synchronisation), so the handle is dropped first: a
+        # second close, or __del__ after a raising close, must not free it again
+        h, self.handle = self.handle, None
+        if h is not None and h.value:
+            cqa_cache_destroy(h)
 
     def __del__(self):
         try:

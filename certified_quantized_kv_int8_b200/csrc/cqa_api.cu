@@ -16,6 +16,7 @@
 
 namespace cqa {
 size_t select_smem_bytes(int G, int nb);
+
 }
 
 using namespace cqa;
@@ -319,6 +320,7 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   if (c.n_layers < 1 || c.batch < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.max_ctx < 1)
     return CQA_ERR_INVALID_ARG;
   if (c.head_dim != 64 && c.head_dim != 128) return CQA_ERR_INVALID_ARG;
+  if (c.meta_fp16 != 0 && c.meta_fp16 != 1) return CQA_ERR_INVALID_ARG;
   if (c.n_q_heads % c.n_kv_heads) return CQA_ERR_INVALID_ARG;
   const int G = c.n_q_heads / c.n_kv_heads;
   if (!(G == 1 || G == 2 || G == 4 || G == 8) || (c.head_dim == 64 && G == 8))
@@ -364,9 +366,10 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   };
   const Strides& st = cc->st;
   const size_t o_kc = take(units * st.kcodes);
-  const size_t o_ks = take(units * st.kscale * 4);
+  const size_t mby = c.meta_fp16 ? 2 : 4;  // bytes of one metadata value
+  const size_t o_ks = take(units * st.kscale * mby);
   const size_t o_vc = take(units * st.vcodes);
-  const size_t o_vm = take(units * st.vmeta * 4);
+  const size_t o_vm = take(units * st.vmeta * mby);
   const size_t o_eta = take(units * st.eta * 4);
   const size_t o_vr = take(units * st.vrange * 4);
   const size_t o_kr = take(units * st.res * 2);
@@ -401,6 +404,9 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->t.kscale = (float*)(bp + o_ks);
   cc->t.vcodes = (uint8_t*)(bp + o_vc);
   cc->t.vmeta = (float*)(bp + o_vm);
+  cc->t.kscale_h = (__half*)(bp + o_ks);
+  cc->t.vmeta_h = (__half*)(bp + o_vm);
+  cc->t.meta16 = c.meta_fp16;
   cc->t.eta = (float*)(bp + o_eta);
   cc->t.vrange = (float*)(bp + o_vr);
   cc->t.kres = (__half*)(bp + o_kr);
@@ -748,9 +754,15 @@ int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t b
   int parts = 1;
   switch (what) {
     case CQA_EXPORT_KCODES: srcs[0] = (const char*)cc->t.kcodes; stride = st.kcodes; break;
-    case CQA_EXPORT_KSCALE: srcs[0] = (const char*)cc->t.kscale; stride = st.kscale * 4; break;
+    case CQA_EXPORT_KSCALE:
+      srcs[0] = (const char*)cc->t.kscale;
+      stride = st.kscale * (cc->t.meta16 ? 2 : 4);
+      break;
     case CQA_EXPORT_VCODES: srcs[0] = (const char*)cc->t.vcodes; stride = st.vcodes; break;
-    case CQA_EXPORT_VMETA: srcs[0] = (const char*)cc->t.vmeta; stride = st.vmeta * 4; break;
+    case CQA_EXPORT_VMETA:
+      srcs[0] = (const char*)cc->t.vmeta;
+      stride = st.vmeta * (cc->t.meta16 ? 2 : 4);
+      break;
     case CQA_EXPORT_ETA: srcs[0] = (const char*)cc->t.eta; stride = st.eta * 4; break;
     case CQA_EXPORT_VRANGE: srcs[0] = (const char*)cc->t.vrange; stride = st.vrange * 4; break;
     case CQA_EXPORT_RESIDUAL:
@@ -799,6 +811,14 @@ int64_t cqa_debug_export(cqa_cache* cc, int layer, int what, void* dst, size_t b
         if (per_unit > sealed &&
             cudaMemcpy(dp + sealed, rs, per_unit - sealed, cudaMemcpyDeviceToHost) != cudaSuccess)
           return CQA_ERR_CUDA;
+      } else if (cc->t.meta16 && (what == CQA_EXPORT_KSCALE || what == CQA_EXPORT_VMETA)) {
+        // binary16 metadata: copy the halves, widen them to float32 (exact)
+        const size_t n = per_unit / 4;
+        std::vector<__half> tmp(n);
+        if (n && cudaMemcpy(tmp.data(), sp, n * 2, cudaMemcpyDeviceToHost) != cudaSuccess)
+          return CQA_ERR_CUDA;
+        float* fd = (float*)dp;
+        for (size_t i = 0; i < n; ++i) fd[i] = __half2float(tmp[i]);
       } else if (cudaMemcpy(dp, sp, per_unit, cudaMemcpyDeviceToHost) != cudaSuccess) {
         return CQA_ERR_CUDA;
       }

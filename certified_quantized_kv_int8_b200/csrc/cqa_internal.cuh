@@ -6,6 +6,8 @@
 //   kscale fp32  [nbm][d]            per (block, channel) key scale
 //   vcodes uint8 [nbm][64][d/2]      INT4 pairs, channel 2j in the low nibble
 //   vmeta  fp32  [nbm][64][d/32][2]  per (token, group): scale, offset
+//   (kscale and vmeta are binary16 instead when the cache stores its
+//   metadata in half precision: Tier1::meta16)
 //   eta    fp32  [nbm]               per-block max INT4 reconstruction error
 //   vrange fp32  [2][d]              running per-channel value min and max
 //   kres, vres fp16 [64][d]          the residual (unsealed) block, exact
@@ -40,9 +42,12 @@ constexpr uint8_t DENSE_LATE = 0x80;
 
 struct Tier1 {
   int8_t* kcodes;
-  float* kscale;
+  float* kscale;     // float32 metadata (meta16 = 0)
   uint8_t* vcodes;
   float* vmeta;
+  __half* kscale_h;  // the same arrays as binary16 (meta16 = 1)
+  __half* vmeta_h;
+  int meta16;        // 1: key scales and value scale/offset stored as binary16
   float* eta;
   float* vrange;
   __half* kres;

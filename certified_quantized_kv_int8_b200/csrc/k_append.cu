@@ -16,6 +16,10 @@
 //   eta_b  max over the block of |v - v_hat|
 // Every step is one IEEE float32 operation (explicit _rn intrinsics, never
 // contracted into an FMA), so codes and annotations are reproducible bit for bit.
+// With binary16 metadata (Tier1::meta16) both scales are rounded up to
+// binary16 (__float2half_ru) before the codes are taken against them, so no
+// code is clamped and the stored scale bounds the rounding error; the value
+// offset, the min of binary16 inputs, is stored exactly.
 #include "cqa_internal.cuh"
 
 namespace cqa {
@@ -84,7 +88,8 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float a = 0.f;
     for (int tk = 0; tk < BLK; ++tk) a = fmaxf(a, fabsf(__half2float(ks[tk * D + c])));
-    sc[c] = __fdiv_rn(a, 127.0f);
+    const float s = __fdiv_rn(a, 127.0f);
+    sc[c] = t.meta16 ? __half2float(__float2half_ru(s)) : s;
   }
   __syncthreads();
 
@@ -104,12 +109,17 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
     }
     reinterpret_cast<uint32_t*>(kc)[e] = w;
   }
-  float* ksc = t.kscale + u * st.kscale + (size_t)j * D;
-  for (int c = threadIdx.x; c < D; c += blockDim.x) ksc[c] = sc[c];
+  if (t.meta16) {
+    __half* ksc = t.kscale_h + u * st.kscale + (size_t)j * D;
+    for (int c = threadIdx.x; c < D; c += blockDim.x) ksc[c] = __float2half_rn(sc[c]);  // exact
+  } else {
+    float* ksc = t.kscale + u * st.kscale + (size_t)j * D;
+    for (int c = threadIdx.x; c < D; c += blockDim.x) ksc[c] = sc[c];
+  }
 
   // values: one thread per (token, group)
   uint8_t* vc = t.vcodes + u * st.vcodes + (size_t)j * BLK * (D / 2);
-  float* vm = t.vmeta + u * st.vmeta + (size_t)j * BLK * NG * 2;
+  const size_t vm0 = u * st.vmeta + (size_t)j * BLK * NG * 2;
   float emax = 0.f;
   for (int e = threadIdx.x; e < BLK * NG; e += blockDim.x) {
     const int tk = e / NG, gi = e % NG;
@@ -120,7 +130,8 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
       lo = fminf(lo, x);
       hi = fmaxf(hi, x);
     }
-    const float s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    float s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    if (t.meta16) s = __half2float(__float2half_ru(s));
     uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int i = 0; i < VG; ++i) {
@@ -136,8 +147,14 @@ __global__ void __launch_bounds__(256) seal_kernel(Tier1 t, Strides st, int unit
     }
     *reinterpret_cast<uint4*>(vc + (size_t)tk * (D / 2) + gi * (VG / 2)) =
         make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    vm[(tk * NG + gi) * 2] = s;
-    vm[(tk * NG + gi) * 2 + 1] = lo;
+    const size_t mi = vm0 + (size_t)(tk * NG + gi) * 2;
+    if (t.meta16) {
+      t.vmeta_h[mi] = __float2half_rn(s);       // exact: s was rounded to binary16
+      t.vmeta_h[mi + 1] = __float2half_rn(lo);  // exact: the min of binary16 inputs
+    } else {
+      t.vmeta[mi] = s;
+      t.vmeta[mi + 1] = lo;
+    }
   }
   atomicMax(&eta_bits, __float_as_int(emax));  // emax >= 0: int order = float order
   __syncthreads();

@@ -254,8 +254,9 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
       if (need_i4) {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(
             t.vcodes + u * st.vcodes + ((size_t)j * BLK + tt) * (D / 2) + cl * 4);
-        meta = *reinterpret_cast<const float2*>(
-            t.vmeta + u * st.vmeta + (((size_t)j * BLK + tt) * NG + (cl * 8) / VG) * 2);
+        const size_t mi = u * st.vmeta + (((size_t)j * BLK + tt) * NG + (cl * 8) / VG) * 2;
+        meta = t.meta16 ? __half22float2(*reinterpret_cast<const __half2*>(t.vmeta_h + mi))
+                        : *reinterpret_cast<const float2*>(t.vmeta + mi);
         u4x8_to_f2(w, cf);
       }
 #pragma unroll

@@ -63,14 +63,35 @@ __host__ __device__ __forceinline__ int naive_cap(int nb, int max_chunks) {
   return c < max_chunks - 1 ? c : max_chunks - 1;
 }
 
-template <int D>
+template <int D, bool MH>
 struct NaiveLayout {
-  static constexpr int KB = BLK * D;              // INT8 key codes
-  static constexpr int SB = 4 * D;                // key scales
-  static constexpr int VB = BLK * D / 2;          // INT4 value codes
-  static constexpr int MB = BLK * (D / VG) * 8;   // value scale/offset
+  static constexpr int MBY = MH ? 2 : 4;               // bytes of one metadata value
+  static constexpr int KB = BLK * D;                   // INT8 key codes
+  static constexpr int SB = MBY * D;                   // key scales
+  static constexpr int VB = BLK * D / 2;               // INT4 value codes
+  static constexpr int MB = BLK * (D / VG) * 2 * MBY;  // value scale/offset
   static constexpr int STAGE = KB + SB + VB + MB;
 };
+
+// four key scales, and one (scale, offset) pair, of a stage as floats
+// (binary16 metadata is widened, exactly)
+template <bool MH>
+__device__ __forceinline__ float4 stage_scales4(const unsigned char* sbase, int c) {
+  if constexpr (MH) {
+    const uint2 v = *reinterpret_cast<const uint2*>(sbase + 2 * c);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    return *reinterpret_cast<const float4*>(sbase + 4 * c);
+  }
+}
+
+template <bool MH>
+__device__ __forceinline__ float2 stage_meta(const unsigned char* mbase, int i) {
+  if constexpr (MH) return __half22float2(*reinterpret_cast<const __half2*>(mbase + 4 * i));
+  else return *reinterpret_cast<const float2*>(mbase + 8 * i);
+}
 
 // channels per lane in the logit step.  The lane holds its channels' scaled
 // queries for every head in registers; 8 channels (16 lanes per token) keep the
@@ -308,13 +329,13 @@ __device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int
   if (tid == 0) sc.cnt[unit] = 0;  // every CTA of this launch has arrived
 }
 
-template <int D, int G>
+template <int D, int G, bool MH>
 __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     naive_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
                  Scratch sc, int trace,
                  float* __restrict__ out, float* __restrict__ e_key, float* __restrict__ e_val,
                  uint8_t* __restrict__ rung) {
-  using LY = NaiveLayout<D>;
+  using LY = NaiveLayout<D, MH>;
   constexpr int NG = D / VG;
   constexpr int CH = NaiveLanes<G>::CH;
   constexpr int CPT = D / CH;        // lanes per token row in the logit step
@@ -378,10 +399,12 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     mbar_arrive_expect_tx(bar, LY::STAGE + 16);
     bulk_g2s(&S.eta[k % NST][0], t.eta + (ei & ~(size_t)3), 16, bar);
     bulk_g2s(dst, t.kcodes + u * st.kcodes + (size_t)j * LY::KB, LY::KB, bar);
-    bulk_g2s(dst + LY::KB, t.kscale + u * st.kscale + (size_t)j * D, LY::SB, bar);
+    const size_t ko = u * st.kscale + (size_t)j * D, mo = u * st.vmeta + (size_t)j * BLK * NG * 2;
+    bulk_g2s(dst + LY::KB, MH ? (const void*)(t.kscale_h + ko) : (const void*)(t.kscale + ko),
+             LY::SB, bar);
     bulk_g2s(dst + LY::KB + LY::SB, t.vcodes + u * st.vcodes + (size_t)j * LY::VB, LY::VB, bar);
-    bulk_g2s(dst + LY::KB + LY::SB + LY::VB, t.vmeta + u * st.vmeta + (size_t)j * BLK * NG * 2,
-             LY::MB, bar);
+    bulk_g2s(dst + LY::KB + LY::SB + LY::VB,
+             MH ? (const void*)(t.vmeta_h + mo) : (const void*)(t.vmeta + mo), LY::MB, bar);
   };
   if (tid == 0)
     for (int k = 0; k < NST; ++k) issue(k);
@@ -414,9 +437,9 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     const int stg = k % NST;
     const bool got = mbar_wait(&S.bar[stg], (uint32_t)((k / NST) & 1), sc.err);
     const unsigned char* sp = dsm + (size_t)stg * LY::STAGE;
-    const float* ks = reinterpret_cast<const float*>(sp + LY::KB);
+    const unsigned char* ks = sp + LY::KB;
     const uint8_t* vc = sp + LY::KB + LY::SB;
-    const float* vm = reinterpret_cast<const float*>(sp + LY::KB + LY::SB + LY::VB);
+    const unsigned char* vm = sp + LY::KB + LY::SB + LY::VB;
 
     // scaled queries of this block and Delta_b (base 2: sum |qs| / 2)
 #pragma unroll
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       if (e - lane < QI) {  // warp-uniform
         const bool act = e < QI;
         const int h = act ? e / (D / 4) : 0, c = act ? 4 * (e % (D / 4)) : 0;
-        const float4 kq = *reinterpret_cast<const float4*>(ks + c);
+        const float4 kq = stage_scales4<MH>(ks, c);
         const float4 qv = *reinterpret_cast<const float4*>(&S.qf[h][c]);
         const float4 r = make_float4(qv.x * kq.x, qv.y * kq.y, qv.z * kq.z, qv.w * kq.w);
         if (act) *reinterpret_cast<float4*>(&S.qs[k & 1][h][c / CH][c % CH]) = r;
@@ -551,10 +574,10 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 #pragma unroll
       for (int li = 0; li < NLI; ++li) {
         const int tok = li * RPW + tr;
-        const float* mrow = vm + ((size_t)(warp * TPW + tok) * NG + dup * GPL) * 2;
+        const int mrow = (warp * TPW + tok) * NG + dup * GPL;
 #pragma unroll
         for (int i = 0; i < GPL; ++i) {
-          const float2 sz = *reinterpret_cast<const float2*>(mrow + 2 * i);
+          const float2 sz = stage_meta<MH>(vm, mrow + i);
           S.ws[warp][tok][dup * GPL + i][pi] = p[li] * sz.x;
           zl[i] = fmaf(p[li], sz.y, zl[i]);
         }
@@ -801,22 +824,31 @@ int naive_chunks(const DecodeShape& sh, int max_chunks) {
   return w;
 }
 
-template <int D, int G>
-cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
-                    const __half* q, const Scratch& sc, float* out, float* e_key, float* e_val,
-                    uint8_t* rung, int trace, cudaStream_t s) {
+template <int D, int G, bool MH>
+cudaError_t naive_mh(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
+                     const __half* q, const Scratch& sc, float* out, float* e_key, float* e_val,
+                     uint8_t* rung, int trace, cudaStream_t s) {
   const int nch = naive_chunks(sh, sc.max_chunks);
-  const int smem = NST * NaiveLayout<D>::STAGE;
+  const int smem = NST * NaiveLayout<D, MH>::STAGE;
   // the merge keeps (nch + 1) * G weights, G inverse sums and NT float4 partial
   // sums in the stage area, after what the CTAs still hold there
   const size_t merge_floats =
       (size_t)NaiveMergeAt<D, G>::AT + (size_t)(nch + 1) * G + G + 4 + (size_t)NT * 4;
   if (merge_floats * 4 > (size_t)smem) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G>, (int)smem);
+  cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G, MH>, (int)smem);
   if (e != cudaSuccess) return e;
-  naive_kernel<D, G><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(
+  naive_kernel<D, G, MH><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(
       t, st, unit0, sh, q, sc, trace, out, e_key, e_val, rung);
   return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t naive_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
+                    const __half* q, const Scratch& sc, float* out, float* e_key, float* e_val,
+                    uint8_t* rung, int trace, cudaStream_t s) {
+  return t.meta16
+             ? naive_mh<D, G, true>(t, st, unit0, sh, q, sc, out, e_key, e_val, rung, trace, s)
+             : naive_mh<D, G, false>(t, st, unit0, sh, q, sc, out, e_key, e_val, rung, trace, s);
 }
 
 }  // namespace

@@ -44,12 +44,25 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr int SCORE_CTAS_PER_SM = 5;  // grid target: resident CTAs per SM
 
-template <int D>
+template <int D, bool MH>
 struct ScoreLayout {
-  static constexpr int KB = BLK * D;  // INT8 key codes
-  static constexpr int SB = 4 * D;    // key scales
+  static constexpr int KB = BLK * D;          // INT8 key codes
+  static constexpr int SB = (MH ? 2 : 4) * D;  // key scales (binary16 or float32)
   static constexpr int STAGE = KB + SB;
 };
+
+// four key scales of the stage as floats
+template <bool MH>
+__device__ __forceinline__ float4 load_scales4(const unsigned char* sbase, int c) {
+  if constexpr (MH) {
+    const uint2 v = *reinterpret_cast<const uint2*>(sbase + 2 * c);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    return *reinterpret_cast<const float4*>(sbase + 4 * c);
+  }
+}
 
 __device__ __forceinline__ float swarp_max(float x) {
 #pragma unroll
@@ -93,11 +106,11 @@ struct ScoreSmem {
   uint64_t bar[NST];
 };
 
-template <int D, int G>
+template <int D, int G, bool MH>
 __global__ void __launch_bounds__(NT, 5)
     score_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
                  Scratch sc) {
-  using LY = ScoreLayout<D>;
+  using LY = ScoreLayout<D, MH>;
   constexpr int CPT = D / CH;     // lanes per token row
   constexpr int RPW = 32 / CPT;   // rows per warp instruction
   constexpr int NLI = TPW / RPW;  // logit iterations per block
@@ -150,7 +163,9 @@ __global__ void __launch_bounds__(NT, 5)
     uint64_t* bar = &S.bar[k % NST];
     mbar_arrive_expect_tx(bar, LY::STAGE);
     bulk_g2s(dst, t.kcodes + u * st.kcodes + (size_t)j * LY::KB, LY::KB, bar);
-    bulk_g2s(dst + LY::KB, t.kscale + u * st.kscale + (size_t)j * D, LY::SB, bar);
+    const void* ksrc = MH ? (const void*)(t.kscale_h + u * st.kscale + (size_t)j * D)
+                          : (const void*)(t.kscale + u * st.kscale + (size_t)j * D);
+    bulk_g2s(dst + LY::KB, ksrc, LY::SB, bar);
   };
   if (tid == 0)
     for (int k = 0; k < NST; ++k) issue(k);
@@ -183,7 +198,7 @@ __global__ void __launch_bounds__(NT, 5)
     const int stg = k % NST;
     const bool got = mbar_wait(&S.bar[stg], (uint32_t)((k / NST) & 1), sc.err);
     const unsigned char* sp = dsm + (size_t)stg * LY::STAGE;
-    const float* ks = reinterpret_cast<const float*>(sp + LY::KB);
+    const unsigned char* ks = sp + LY::KB;
 
     // scaled queries of this block and Delta_b = sum |qs| / 2
 #pragma unroll
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(NT, 5)
       if (e - lane < QI) {  // warp-uniform
         const bool act = e < QI;
         const int h = act ? e / (D / 4) : 0, c = act ? 4 * (e % (D / 4)) : 0;
-        const float4 kq = *reinterpret_cast<const float4*>(ks + c);
+        const float4 kq = load_scales4<MH>(ks, c);
         const float4 qv = *reinterpret_cast<const float4*>(&S.qf[h][c]);
         const float4 r = make_float4(qv.x * kq.x, qv.y * kq.y, qv.z * kq.z, qv.w * kq.w);
         if (act) *reinterpret_cast<float4*>(&S.qs[k & 1][h][c / CH][c % CH]) = r;
@@ -379,15 +394,22 @@ int score_chunks(const DecodeShape& sh) {
   return w;
 }
 
+template <int D, int G, bool MH>
+cudaError_t launch_score_mh(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
+                            const __half* q, const Scratch& sc, cudaStream_t s) {
+  const int nch = score_chunks(sh);
+  const int smem = NST * ScoreLayout<D, MH>::STAGE;
+  cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G, MH>, (int)smem);
+  if (e != cudaSuccess) return e;
+  score_kernel<D, G, MH><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc);
+  return cudaGetLastError();
+}
+
 template <int D, int G>
 cudaError_t launch_score_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                            const __half* q, const Scratch& sc, cudaStream_t s) {
-  const int nch = score_chunks(sh);
-  const int smem = NST * ScoreLayout<D>::STAGE;
-  cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G>, (int)smem);
-  if (e != cudaSuccess) return e;
-  score_kernel<D, G><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc);
-  return cudaGetLastError();
+  return t.meta16 ? launch_score_mh<D, G, true>(t, st, unit0, sh, q, sc, s)
+                  : launch_score_mh<D, G, false>(t, st, unit0, sh, q, sc, s);
 }
 
 }  // namespace

@@ -68,6 +68,13 @@ typedef struct cqa_config {
   int32_t head_dim;   /* 64 or 128 */
   int32_t max_ctx;    /* token capacity per (layer, batch row), >= 1 */
   int32_t device;     /* CUDA device ordinal the cache lives on */
+  int32_t meta_fp16;  /* Tier-1 metadata precision (Methodology §1 leaves it open):
+                         0: key scales and value scale/offset in float32 (232 B per token
+                         and kv head at head_dim 128); 1: in binary16 (212 B): each
+                         scale is rounded up to binary16 before the codes are taken
+                         against it, so no code clamps and the stored scale still bounds
+                         the rounding error; the value offset (a group min of binary16
+                         inputs) is stored exactly */
 } cqa_config;
 
 /* Largest rank_r a decode accepts (CQA_ERR_INVALID_ARG above it). */
@@ -187,7 +194,8 @@ int cqa_dense_reference(cqa_cache* cache, int layer, const void* q_fp16, float* 
  * (batch row, kv head) takes its own row's extent (its nb, length % 64 and
  * length), and the units follow one another in [batch][n_kv_heads] order:
  *   CQA_EXPORT_KCODES   int8  [batch][n_kv_heads][nb][64][d]
- *   CQA_EXPORT_KSCALE   fp32  [batch][n_kv_heads][nb][d]
+ *   CQA_EXPORT_KSCALE   fp32  [batch][n_kv_heads][nb][d]  (binary16 metadata is
+ *                       exported widened to fp32, exactly, like VMETA)
  *   CQA_EXPORT_VCODES   uint8 [batch][n_kv_heads][nb][64][d/2]  (channel 2j low nibble)
  *   CQA_EXPORT_VMETA    fp32  [batch][n_kv_heads][nb][64][d/32][2]  (scale, offset)
  *   CQA_EXPORT_ETA      fp32  [batch][n_kv_heads][nb]

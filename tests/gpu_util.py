@@ -48,10 +48,10 @@ def fill_cache(cache, w, layers, ctx, chunks=None, device="cuda"):
     torch.cuda.synchronize()
 
 
-def oracle_units(w, layer, b, ctx):
+def oracle_units(w, layer, b, ctx, fp16_meta=False):
     from oracle import build_unit
     K, V = sk.kv_layer(w, layer, 0, ctx, device="cpu")
-    return [build_unit(K[b, g].numpy(), V[b, g].numpy()) for g in range(w.n_kv_heads)]
+    return [build_unit(K[b, g].numpy(), V[b, g].numpy(), fp16_meta) for g in range(w.n_kv_heads)]
 
 
 def oracle_thresholds(th):

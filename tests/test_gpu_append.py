@@ -34,7 +34,7 @@ def test_generator_identical_on_device():
         assert torch.equal(qc, sk.queries(w, 0, 5, "cuda").cpu())
 
 
-def _check_unit_arrays(cache, layer, w, wl, ctx):
+def _check_unit_arrays(cache, layer, w, wl, ctx, fp16_meta=False):
     from oracle import build_unit, pack_int4
     kc = cache.export(layer, 0)
     ks = cache.export(layer, 1)
@@ -47,7 +47,7 @@ def _check_unit_arrays(cache, layer, w, wl, ctx):
     K, V = sk.kv_layer(w, wl, 0, ctx, "cpu")
     for b in range(w.batch):
         for g in range(w.n_kv_heads):
-            u = build_unit(K[b, g].numpy(), V[b, g].numpy())
+            u = build_unit(K[b, g].numpy(), V[b, g].numpy(), fp16_meta)
             np.testing.assert_array_equal(kc[b, g], u["kcodes"])
             np.testing.assert_array_equal(ks[b, g], u["kscale"])
             np.testing.assert_array_equal(vc[b, g], pack_int4(u["vcodes"]))
@@ -80,6 +80,18 @@ def test_append_d128_bit_exact(cqa, name, ctx):
     with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx) as cache:
         fill_cache(cache, w, [0], ctx, chunks=[500, 3000, 17])
         _check_unit_arrays(cache, 0, w, 0, ctx)
+
+
+@pytest.mark.parametrize("name,ctx,chunks", [("tiny", 1024 + 37, [1, 63, 64, 100, 1, 700]),
+                                             ("llama8b_8k_1layer", 4096 + 45, None),
+                                             ("llama8b_64k_b4_t3values", 2048 + 64, [500, 17])])
+def test_append_fp16_meta_bit_exact(cqa, name, ctx, chunks):
+    """Binary16 metadata: scales rounded up, codes taken against them, offsets exact."""
+    w = sk.WORKLOADS[name]
+    with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx,
+                   meta_fp16=True) as cache:
+        fill_cache(cache, w, [0], ctx, chunks=chunks)
+        _check_unit_arrays(cache, 0, w, 0, ctx, fp16_meta=True)
 
 
 def test_append_errors(cqa):

@@ -22,17 +22,18 @@ def cqa():
     return m
 
 
-def _check(cqa, w, ctx, th, layers=(0,), step=0, label=""):
+def _check(cqa, w, ctx, th, layers=(0,), step=0, label="", fp16_meta=False):
     from oracle import decode
     log = TieLog()
-    with cqa.Cache(len(layers), w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx) as cache:
+    with cqa.Cache(len(layers), w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, ctx,
+                   meta_fp16=fp16_meta) as cache:
         fill_cache(cache, w, list(layers), ctx)
         for i, layer in enumerate(layers):
             q = sk.queries(w, layer, step, "cuda")
             res = run_decode(cache, i, q, th)
             qc = q.cpu().numpy()
             for b in range(w.batch):
-                units = oracle_units(w, layer, b, ctx)
+                units = oracle_units(w, layer, b, ctx, fp16_meta)
                 ora = decode(qc[b], units, oracle_thresholds(th))
                 compare_decode(row(res, b), ora, oracle_thresholds(th), w.group, log,
                                label=f"{label} layer {layer} b {b}")
@@ -73,6 +74,17 @@ def test_decode_short_contexts(cqa, ctx, naive):
     w = sk.WORKLOADS["tiny"]
     th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.7, "naive": naive})
     _check(cqa, w, ctx, th, label=f"ctx{ctx}{' naive' if naive else ''}")
+
+
+@pytest.mark.parametrize("name,ctx", [("tiny", 1024 + 19), ("llama8b_8k_1layer", 8192 + 21),
+                                      ("llama8b_64k_b4_t3values", 4096 + 5)])
+@pytest.mark.parametrize("naive", [False, True])
+def test_decode_fp16_meta(cqa, name, ctx, naive):
+    """Binary16 Tier-1 metadata through the certified and the INT8/INT4 paths."""
+    w = sk.WORKLOADS[name]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.8, "naive": naive})
+    log = _check(cqa, w, ctx, th, label=f"fp16 meta {name}", fp16_meta=True)
+    assert len(log.entries) <= 2
 
 
 def test_decode_llama8b_8k(cqa):
