@@ -33,10 +33,12 @@
 //     and each level halves the values in flight;
 //   * logits are kept in base 2 (queries pre-scaled by log2 e) so every
 //     exponential is one exp2;
-//   * INT4 codes become floats by masking a nibble into the mantissa of 2^23
-//     (nibbles 0-4 of a word in place, 5-7 after one shift) and one packed
-//     subtraction; each nibble then carries a power-of-two factor (16^k, or
-//     16^(k-5)) that is divided out of its accumulator once per chunk (exact);
+//   * INT4 codes become floats without an FP32 operation: each nibble is
+//     shifted under the exponent of 16 (even channels, value 16 + n) or of
+//     256 (odd channels, value 256 + n) with one LOP3; the constant is removed
+//     once per chunk with the per-group sum of weights the softmax lanes keep
+//     (Sum w (C + n) - C Sum w), which leaves the FP32 pipe to the
+//     multiply-adds;
 //   * the value scale is folded into the attention weight per (token, group,
 //     head) by the softmax lanes, which also accumulate the offset term.
 #include "bulk_pipe.cuh"
@@ -125,21 +127,24 @@ __device__ __forceinline__ void s8x4_f2(uint32_t w, float2& a, float2& b) {
                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653))), off);
 }
 
-// eight INT4 codes (nibble k = channel k) -> c[k/2] = (n_k * 16^e_k, n_k+1 * 16^e_k+1)
-// with e = 0,1,2,3,4,0,1,2
-__device__ __forceinline__ void u4x8_scaled(uint32_t w, float2 (&c)[4]) {
-  const uint32_t m = 0x4B000000u;
-  const uint32_t h = w >> 20;
-  const float2 off = make_float2(-8388608.0f, -8388608.0f);
-  c[0] = __fadd2_rn(make_float2(__uint_as_float((w & 0xFu) | m),
-                                __uint_as_float((w & 0xF0u) | m)), off);
-  c[1] = __fadd2_rn(make_float2(__uint_as_float((w & 0xF00u) | m),
-                                __uint_as_float((w & 0xF000u) | m)), off);
-  c[2] = __fadd2_rn(make_float2(__uint_as_float((w & 0xF0000u) | m),
-                                __uint_as_float((h & 0xFu) | m)), off);
-  c[3] = __fadd2_rn(make_float2(__uint_as_float((h & 0xF0u) | m),
-                                __uint_as_float((h & 0xF00u) | m)), off);
+// eight INT4 codes (nibble k = channel k) -> floats C_k + n_k without an FP32
+// operation: even nibbles are shifted to mantissa bits 19-22 under the exponent
+// of 16 (value 16 + n), odd ones to bits 15-18 under the exponent of 256
+// (value 256 + n); c[p] = (channel 2p, channel 2p + 1)
+__device__ __forceinline__ void u4x8_biased(uint32_t w, float2 (&c)[4]) {
+  const uint32_t s0 = w << 19;  // n0 -> 19
+  const uint32_t s1 = w << 11;  // n1 -> 15, n2 -> 19
+  const uint32_t s2 = w << 3;   // n3 -> 15, n4 -> 19
+  const uint32_t s3 = w >> 5;   // n5 -> 15, n6 -> 19
+  const uint32_t s4 = w >> 13;  // n7 -> 15
+  constexpr uint32_t E16 = 0x41800000u, E256 = 0x43800000u;
+  constexpr uint32_t M19 = 0xFu << 19, M15 = 0xFu << 15;
+  c[0] = make_float2(__uint_as_float((s0 & M19) | E16), __uint_as_float((s1 & M15) | E256));
+  c[1] = make_float2(__uint_as_float((s1 & M19) | E16), __uint_as_float((s2 & M15) | E256));
+  c[2] = make_float2(__uint_as_float((s2 & M19) | E16), __uint_as_float((s3 & M15) | E256));
+  c[3] = make_float2(__uint_as_float((s3 & M19) | E16), __uint_as_float((s4 & M15) | E256));
 }
+
 
 // 2^x by the hardware approximation (relative error about 2^-22; flushes
 // results below 2^-126 to zero, which only drops weights that small)
@@ -149,12 +154,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 16^-e of nibble k (see u4x8_scaled)
-__device__ __forceinline__ float nib_unscale(int k) {
-  const int e = k < 5 ? k : k - 5;
-  return __int_as_float((127 - 4 * e) << 23);
-}
-
 // float offsets in the stage area where the merge of a unit's partials starts:
 // after the residual block's logits and statistics and after the per-warp
 // states, which a CTA may both hold there (multiples of 4 floats, so the
@@ -162,7 +161,7 @@ __device__ __forceinline__ float nib_unscale(int k) {
 template <int D, int G>
 struct NaiveMergeAt {
   static constexpr int RES = (G * BLK + 2 * G + 3) / 4 * 4;
-  static constexpr int MAIN = NW * G * (D + D / VG + 3);
+  static constexpr int MAIN = NW * G * (D + 2 * (D / VG) + 3);
   static constexpr int AT = RES > MAIN ? RES : MAIN;
   static_assert(MAIN % 4 == 0, "alignment");
 };
@@ -420,14 +419,14 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
   const int cl = lane % LPT, ts = lane / LPT;  // P.V step: channel slice, row
   const int gq = cl * 8 / VG;
 
-  float2 acc[G][4];  // P.V accumulators, channel 8*cl + k carries 16^e_k
+  float2 acc[G][4];  // P.V accumulators, channel 8*cl + k carries C = 16 (k even) or 256 (k odd)
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
-  float zl[GPL];  // offset term: sum of weight * value offset, per owned group of head pi
+  float zl[GPL], wl[GPL];  // offset term and weight sum, per owned group of head pi
 #pragma unroll
-  for (int i = 0; i < GPL; ++i) zl[i] = 0.f;
+  for (int i = 0; i < GPL; ++i) zl[i] = wl[i] = 0.f;
   float mrun = -INFINITY, lrun = 0.f, erun = 0.f;  // running state of head pi (base 2)
 
   bool ok = true;
@@ -570,7 +569,10 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     // value scale folded into the weights; offset term accumulated here
     if (dup * GPL < NG) {
 #pragma unroll
-      for (int i = 0; i < GPL; ++i) zl[i] *= alpha;
+      for (int i = 0; i < GPL; ++i) {
+        zl[i] *= alpha;
+        wl[i] *= alpha;
+      }
 #pragma unroll
       for (int li = 0; li < NLI; ++li) {
         const int tok = li * RPW + tr;
@@ -578,7 +580,9 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 #pragma unroll
         for (int i = 0; i < GPL; ++i) {
           const float2 sz = stage_meta<MH>(vm, mrow + i);
-          S.ws[warp][tok][dup * GPL + i][pi] = p[li] * sz.x;
+          const float wv = p[li] * sz.x;
+          S.ws[warp][tok][dup * GPL + i][pi] = wv;
+          wl[i] += wv;
           zl[i] = fmaf(p[li], sz.y, zl[i]);
         }
       }
@@ -614,7 +618,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
         for (int h = 0; h < G; ++h) wsv[h] = S.ws[warp][tok][gq][h];
       }
       float2 cf[4];
-      u4x8_scaled(w, cf);
+      u4x8_biased(w, cf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float2 ww = make_float2(wsv[h], wsv[h]);
@@ -648,8 +652,8 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 
   // ---- merge the four warps' states ----
   float* ow = reinterpret_cast<float*>(dsm);  // [NW][G][D] unscaled P.V of each warp
-  float* zw = ow + NW * G * D;                // [NW][G][NG] offset terms
-  float* mw = zw + NW * G * NG;               // [NW][G][3] m, l, e
+  float* zw = ow + NW * G * D;                // [NW][G][NG][2] offset term minus C * weight sum
+  float* mw = zw + NW * G * NG * 2;           // [NW][G][3] m, l, e
 #pragma unroll
   for (int m = LPT; m < 32; m <<= 1)
 #pragma unroll
@@ -665,15 +669,22 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         *reinterpret_cast<float2*>(&ow[(warp * G + h) * D + cl * 8 + 2 * i]) =
-            make_float2(acc[h][i].x * nib_unscale(2 * i), acc[h][i].y * nib_unscale(2 * i + 1));
+            acc[h][i];
   }
 #pragma unroll
   for (int m = CPT; m < 32; m <<= 1)
 #pragma unroll
-    for (int i = 0; i < GPL; ++i) zl[i] += __shfl_xor_sync(0xffffffffu, zl[i], m);
+    for (int i = 0; i < GPL; ++i) {
+      zl[i] += __shfl_xor_sync(0xffffffffu, zl[i], m);
+      wl[i] += __shfl_xor_sync(0xffffffffu, wl[i], m);
+    }
   if (tr == 0 && dup * GPL < NG) {
 #pragma unroll
-    for (int i = 0; i < GPL; ++i) zw[(warp * G + pi) * NG + dup * GPL + i] = zl[i];
+    for (int i = 0; i < GPL; ++i) {
+      // channels of even index carry C = 16, odd ones C = 256
+      zw[((warp * G + pi) * NG + dup * GPL + i) * 2] = zl[i] - 16.f * wl[i];
+      zw[((warp * G + pi) * NG + dup * GPL + i) * 2 + 1] = zl[i] - 256.f * wl[i];
+    }
   }
   if (owner) {
     mw[(warp * G + pi) * 3 + 0] = mrun;
@@ -691,7 +702,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
         const float f = exp2f(mw[(w * G + h) * 3] - M);
-        o = fmaf(f, ow[(w * G + h) * D + c] + zw[(w * G + h) * NG + c / VG], o);
+        o = fmaf(f, ow[(w * G + h) * D + c] + zw[((w * G + h) * NG + c / VG) * 2 + (c & 1)], o);
       }
     }
     sc.part_o[(pbase + h) * D + c] = o;
