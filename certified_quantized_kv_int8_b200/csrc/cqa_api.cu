@@ -389,7 +389,6 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   const size_t o_ps = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
   const size_t o_err = take(sizeof(int));
   const size_t o_px = take((size_t)c.batch * c.n_kv_heads * max_chunks * G * 3 * 4);
-  const size_t o_cnt = take((size_t)c.batch * c.n_kv_heads * sizeof(int));
   const size_t o_dcnt = take((size_t)c.batch * 2 * sizeof(int));
   const size_t o_lens = take((size_t)c.n_layers * c.batch * sizeof(int32_t));
   void* base = nullptr;
@@ -425,7 +424,6 @@ int cqa_cache_create(const cqa_config* cfg, cqa_cache** out) {
   cc->sc.part_s = (float*)(bp + o_ps);
   cc->sc.err = (int*)(bp + o_err);
   cc->sc.part_x = (float*)(bp + o_px);
-  cc->sc.cnt = (int*)(bp + o_cnt);
   cc->sc.dcnt = (int*)(bp + o_dcnt);
   cc->lens_dev = (int32_t*)(bp + o_lens);
   cc->sc.ls = ls;
@@ -680,6 +678,10 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
       return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung,
                           trace != nullptr, s);
     });
+    if (e == cudaSuccess)
+      e = run_phase(cc, CQA_PHASE_NAIVE_COMBINE, s, 1, [&] {
+        return launch_naive_combine(sh, cc->sc, out, e_key, e_val, rung, s);
+      });
     if (e != cudaSuccess) return CQA_ERR_CUDA;
     if (trace) return copy_trace(cc, sh, trace, s);
     return CQA_OK;
@@ -837,9 +839,7 @@ int cqa_device_status(cqa_cache* cc, int32_t* status) {
     return CQA_ERR_CUDA;
   if (v) {
     // a kernel that gave up may have left its arrival counters short of zero
-    const size_t units = (size_t)cc->cfg.batch * cc->cfg.n_kv_heads;
     if (cudaMemset(cc->sc.err, 0, sizeof(int)) != cudaSuccess ||
-        cudaMemset(cc->sc.cnt, 0, units * sizeof(int)) != cudaSuccess ||
         cudaMemset(cc->sc.dcnt, 0, (size_t)cc->cfg.batch * 2 * sizeof(int)) != cudaSuccess)
       return CQA_ERR_CUDA;
   }

@@ -91,7 +91,6 @@ struct Scratch {
   int32_t* promo;    // [n_layers * B * Hkv] promoted block count per unit (pinned host, mapped)
   int* err;          // device error word (bit 0: a bounded wait gave up)
   float* part_x;     // [B*Hkv][max_chunks][G][3]  naive pass: (max Delta, residual m, residual l)
-  int* cnt;          // [B*Hkv] naive pass: CTAs of the unit that have finished (0 between calls)
   int* dcnt;         // [B][2] rank check: rung-3 heads, heads done (0 between calls)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
@@ -131,6 +130,34 @@ __host__ __device__ __forceinline__ int unit_ctas(int target, int items, long lo
   return n < 1 ? 1 : (int)n;
 }
 
+// Programmatic dependent launch.  The kernels of a decode step are launched
+// with programmatic stream serialization: a kernel's CTAs may be scheduled
+// while the previous kernel on the stream drains.  Each such kernel first lets
+// its own dependent be scheduled (once all of its CTAs have started), then
+// waits until the previous kernel has completed and its writes are visible,
+// before touching global memory, so only the launch and scheduling latency
+// overlap, never a data dependence.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
 // again only when a launch needs more than already granted: the attribute
 // call may stall the host, so it stays off the per-launch path.
@@ -163,12 +190,15 @@ cudaError_t launch_select(const Tier1& t, const Strides& st, int layer_unit0,
 cudaError_t launch_attend(const Tier1& t, const Strides& st, int layer_unit0,
                           const DecodeShape& sh, const __half* q, const Scratch& sc, int mode,
                           cudaStream_t s);
-// certification off: one streaming pass over Tier 1 whose last CTA per unit
-// merges the partials into the outputs; with `trace` set the pass also writes
-// the per-block ell8, Delta and block flags of the trace
+// certification off: one streaming pass over Tier 1 into split-K partials;
+// with `trace` set the pass also writes the per-block ell8, Delta and block
+// flags of the trace
 cudaError_t launch_naive(const Tier1& t, const Strides& st, int layer_unit0, const DecodeShape& sh,
                          const __half* q, const Scratch& sc, float* out, float* e_key,
                          float* e_val, uint8_t* rung, int trace, cudaStream_t s);
+// the combine of that pass's split-K partials into the outputs, E_key, E_val
+cudaError_t launch_naive_combine(const DecodeShape& sh, const Scratch& sc, float* out,
+                                 float* e_key, float* e_val, uint8_t* rung, cudaStream_t s);
 cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                            float* out, float* e_key, float* e_val, uint8_t* rung,
                            cudaStream_t s);

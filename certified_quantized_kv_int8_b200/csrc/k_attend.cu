@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
                                                          DecodeShape sh,
                                                          const __half* __restrict__ q,
                                                          Scratch sc) {
+  pdl_begin();
   constexpr int LPR = D / 8;              // threads per token row, 8 channels each
   constexpr int RPC = THREADS / LPR;      // rows handled per pass
   constexpr int NPASS = BLK / RPC;        // passes per block
@@ -305,12 +306,11 @@ cudaError_t launch_attend_t(const Tier1& t, const Strides& st, int unit0, const 
                             const __half* q, const Scratch& sc, int mode, cudaStream_t s) {
   dim3 grid(sh.nchunks, sh.B * sh.Hkv);
   if (mode == 0)
-    attend_kernel<D, G, 0><<<grid, THREADS, 0, s>>>(t, st, unit0, sh, q, sc);
+    return launch_pdl(attend_kernel<D, G, 0>, grid, dim3(THREADS), 0, s, t, st, unit0, sh, q, sc);
   else if (mode == 1)
-    attend_kernel<D, G, 1><<<grid, THREADS, 0, s>>>(t, st, unit0, sh, q, sc);
+    return launch_pdl(attend_kernel<D, G, 1>, grid, dim3(THREADS), 0, s, t, st, unit0, sh, q, sc);
   else
-    attend_kernel<D, G, 2><<<grid, THREADS, 0, s>>>(t, st, unit0, sh, q, sc);
-  return cudaGetLastError();
+    return launch_pdl(attend_kernel<D, G, 2>, grid, dim3(THREADS), 0, s, t, st, unit0, sh, q, sc);
 }
 
 }  // namespace

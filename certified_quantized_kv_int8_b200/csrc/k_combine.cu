@@ -57,6 +57,7 @@ __device__ __forceinline__ KI warp_best(KI v) {
 
 __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_thresholds th,
                                                     int need_dense, Scratch sc, int staged) {
+  pdl_begin();
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ KI red[2][DW];
   __shared__ int cnt[DW];
@@ -286,6 +287,7 @@ template <int D, int G>
 __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
                                float* __restrict__ out, float* __restrict__ e_key,
                                float* __restrict__ e_val, uint8_t* __restrict__ rung) {
+  pdl_begin();
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   const int g = h / G, hh = h - g * G;
@@ -321,6 +323,7 @@ template <int D, int G>
 __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
                                      float* __restrict__ out, float* __restrict__ e_key,
                                      float* __restrict__ e_val, uint8_t* __restrict__ rung) {
+  pdl_begin();
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   if (!all_heads && !(sc.dense[row] & DENSE_LATE)) return;
@@ -338,16 +341,15 @@ __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
 template <int D, int G>
 cudaError_t combine_t(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                       float* out, float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  combine_kernel<D, G><<<sh.B * sh.Hq, D, 0, s>>>(sh, th, sc, out, e_key, e_val, rung);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(D), 0, s, sh, th, sc, out, e_key,
+                    e_val, rung);
 }
 
 template <int D, int G>
 cudaError_t dense_combine_t(const DecodeShape& sh, const Scratch& sc, int all_heads, float* out,
                             float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  dense_combine_kernel<D, G><<<sh.B * sh.Hq, D, 0, s>>>(sh, sc, all_heads, out, e_key, e_val,
-                                                        rung);
-  return cudaGetLastError();
+  return launch_pdl(dense_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(D), 0, s, sh, sc,
+                    all_heads, out, e_key, e_val, rung);
 }
 
 }  // namespace
@@ -387,8 +389,8 @@ cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int n
     cudaError_t e = ensure_dynamic_smem((const void*)decide_kernel, smem);
     if (e != cudaSuccess) return e;
   }
-  decide_kernel<<<sh.B * sh.Hq, DT, smem, s>>>(sh, th, need_dense, sc, staged);
-  return cudaGetLastError();
+  return launch_pdl(decide_kernel, dim3(sh.B * sh.Hq), dim3(DT), smem, s, sh, th, need_dense, sc,
+                    staged);
 }
 
 cudaError_t launch_dense_combine(const DecodeShape& sh, const Scratch& sc, int all_heads,

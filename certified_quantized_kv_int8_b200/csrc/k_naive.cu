@@ -1,7 +1,8 @@
 // The INT8/INT4 decode path with certification off: one streaming pass over
 // Tier 1 that scores the INT8 keys, runs the online softmax and accumulates
-// the INT4 values; the last CTA of each (batch row, kv head) to finish merges
-// the split-K partials and reports the outputs, E_key and E_val.
+// the INT4 values into split-K partials, and a combine kernel, launched as a
+// programmatic dependent of the pass, that merges them and reports the
+// outputs, E_key and E_val.
 //
 // Runtime-Certified Bounded-Error Quantized Attention, Experimental Results
 // (the naive INT8/INT4 baseline, without certification) and Methodology §2
@@ -154,16 +155,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// float offsets in the stage area where the merge of a unit's partials starts:
-// after the residual block's logits and statistics and after the per-warp
-// states, which a CTA may both hold there (multiples of 4 floats, so the
-// merge's float4 scratch stays aligned)
+// floats of the stage area a CTA reuses after its last block: the per-warp
+// states of the chunk end, then the residual block's logits and statistics
 template <int D, int G>
-struct NaiveMergeAt {
-  static constexpr int RES = (G * BLK + 2 * G + 3) / 4 * 4;
+struct NaiveScratchFloats {
+  static constexpr int RES = G * BLK + 2 * G;
   static constexpr int MAIN = NW * G * (D + 2 * (D / VG) + 3);
-  static constexpr int AT = RES > MAIN ? RES : MAIN;
-  static_assert(MAIN % 4 == 0, "alignment");
+  static constexpr int N = RES > MAIN ? RES : MAIN;
 };
 
 template <int D, int G>
@@ -177,7 +175,6 @@ struct NaiveSmem {
   float ellp[2][NW][G];            // trace: log2-sum-exp of each warp's tokens of a block
   float dmax[G];
   __align__(16) float eta[NST][4];  // the 16-byte run of eta holding eta_b of each stage's block
-  int last;        // this CTA merges its unit's partials
   uint64_t bar[NST];
 };
 
@@ -187,153 +184,13 @@ __device__ double naive_e_key(double dT, double dA, double m8T) {
   return fmin(tanh(0.5 * dT), m_ub * expm1(2.0 * dT));
 }
 
-// Arrival of one CTA of a (batch row, kv head) unit; the last of its narr
-// CTAs merges the unit's nparts partials (split-K combine; the last part is
-// the residual block's) into the outputs o / L, E_key from the largest Delta
-// and the residual's mass, and E_val = sum of eta-weighted mass / L.  Every CTA of the launch calls this
-// exactly once, also after a failed wait, so the arrival counter returns to
-// zero for the next launch.
-template <int D, int G>
-__device__ void naive_arrive_merge(const DecodeShape& sh, const Scratch& sc, int nparts, int narr,
-                                   int unit, int nb,
-                                   size_t hrow0, float* __restrict__ out,
-                                   float* __restrict__ e_key, float* __restrict__ e_val,
-                                   uint8_t* __restrict__ rung, float* wsm, int* flag) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  __threadfence();  // this thread's partials, before the arrival below
-  __syncthreads();
-  if (tid == 0) *flag = atomicAdd(&sc.cnt[unit], 1) == narr - 1;
-  __syncthreads();
-  if (!*flag) return;
-  __threadfence();
-  const size_t base = (size_t)unit * sc.max_chunks * G;  // partial index of (chunk 0, head 0)
-  float* wt = wsm;                  // [nparts][G] weights exp(m_c - M)
-  float* hs = wsm + nparts * G;     // [G] 1 / L
-  // per head (one warp each): the parts' (m, l, e, max Delta) are loaded in one
-  // round when they fit a lane's registers (up to 32 * PPL parts), else twice
-  constexpr int PPL = 4;  // parts per lane per round
-  for (int h = warp; h < G; h += NW) {
-    float M = -INFINITY, dA = 0.f, ll = 0.f, el = 0.f;
-    float mv[PPL], lv[PPL], ev[PPL];
-    for (int c0 = 0; c0 < nparts; c0 += 32 * PPL) {
-      float dv[PPL];
-#pragma unroll
-      for (int i = 0; i < PPL; ++i) {
-        const int c = c0 + i * 32 + lane;
-        const float* ps = sc.part_s + (base + (size_t)c * G + h) * 3;
-        const bool in = c < nparts;
-        mv[i] = in ? __ldcg(ps) : -INFINITY;
-        lv[i] = in ? __ldcg(ps + 1) : 0.f;
-        ev[i] = in ? __ldcg(ps + 2) : 0.f;
-        dv[i] = in ? __ldcg(&sc.part_x[(base + (size_t)c * G + h) * 3]) : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < PPL; ++i) {
-        M = fmaxf(M, mv[i]);
-        dA = fmaxf(dA, dv[i]);
-      }
-    }
-    M = nwarp_max(M);
-    dA = nwarp_max(dA);
-    for (int c0 = 0; c0 < nparts; c0 += 32 * PPL) {
-      if (nparts > 32 * PPL) {  // the registers hold the last round only: reload
-#pragma unroll
-        for (int i = 0; i < PPL; ++i) {
-          const int c = c0 + i * 32 + lane;
-          const float* ps = sc.part_s + (base + (size_t)c * G + h) * 3;
-          const bool in = c < nparts;
-          mv[i] = in ? __ldcg(ps) : -INFINITY;
-          lv[i] = in ? __ldcg(ps + 1) : 0.f;
-          ev[i] = in ? __ldcg(ps + 2) : 0.f;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < PPL; ++i) {
-        const int c = c0 + i * 32 + lane;
-        const float w = mv[i] == -INFINITY ? 0.f : expf(mv[i] - M);
-        if (c < nparts) wt[c * G + h] = w;
-        ll = fmaf(lv[i], w, ll);
-        el = fmaf(ev[i], w, el);
-      }
-    }
-    const float L = nwarp_sum(ll), E = nwarp_sum(el);
-    if (lane == 0) {
-      const size_t row = hrow0 + h;
-      hs[h] = 1.f / L;
-      // the residual CTA (the last part) holds the residual's own statistics
-      const float* px = sc.part_x + (base + (size_t)(nparts - 1) * G + h) * 3;
-      const float mr = __ldcg(px + 1);
-      const double mres = mr == -INFINITY ? 0.0 : (double)__ldcg(px + 2) * exp((double)mr - M) / L;
-      const float ek = nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
-      e_key[row] = ek;
-      e_val[row] = E / L;
-      rung[row] = 0;
-      sc.ekey[row] = ek;
-      sc.hflags[row] = 0;
-      sc.kstar[row] = 0;
-      sc.dense[row] = 0;
-    }
-  }
-  __syncthreads();
-  // outputs: float4 items (head, 4 channels); PS threads split the parts of an item
-  constexpr int NI = G * D / 4;
-  constexpr int PS = NI >= NT ? 1 : NT / NI;
-  float4* red = reinterpret_cast<float4*>(wsm + nparts * G + G + (4 - (nparts * G + G) % 4) % 4);
-  for (int it = tid; it < NI * PS; it += NT) {
-    const int item = it % NI, sl = it / NI;
-    const int h = item / (D / 4), c4 = item % (D / 4);
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = sl; c0 < nparts; c0 += 16 * PS) {
-      float4 v[16];
-      float wv[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = c0 + i * PS;
-        const bool in = c < nparts;
-        v[i] = in ? __ldcg(reinterpret_cast<const float4*>(
-                        sc.part_o + (base + (size_t)c * G + h) * D) + c4)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-        wv[i] = in ? wt[c * G + h] : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        o.x = fmaf(v[i].x, wv[i], o.x);
-        o.y = fmaf(v[i].y, wv[i], o.y);
-        o.z = fmaf(v[i].z, wv[i], o.z);
-        o.w = fmaf(v[i].w, wv[i], o.w);
-      }
-    }
-    if (PS == 1) {
-      const float il = hs[h];
-      reinterpret_cast<float4*>(out + (hrow0 + h) * D)[c4] =
-          make_float4(o.x * il, o.y * il, o.z * il, o.w * il);
-    } else {
-      red[it] = o;
-    }
-  }
-  if (PS > 1) {
-    __syncthreads();
-    for (int item = tid; item < NI; item += NT) {
-      const int h = item / (D / 4), c4 = item % (D / 4);
-      float4 o = red[item];
-      for (int sl = 1; sl < PS; ++sl) {
-        const float4 t2 = red[sl * NI + item];
-        o.x += t2.x; o.y += t2.y; o.z += t2.z; o.w += t2.w;
-      }
-      const float il = hs[h];
-      reinterpret_cast<float4*>(out + (hrow0 + h) * D)[c4] =
-          make_float4(o.x * il, o.y * il, o.z * il, o.w * il);
-    }
-  }
-  if (tid == 0) sc.cnt[unit] = 0;  // every CTA of this launch has arrived
-}
-
 template <int D, int G, bool MH>
 __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     naive_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
                  Scratch sc, int trace,
                  float* __restrict__ out, float* __restrict__ e_key, float* __restrict__ e_val,
                  uint8_t* __restrict__ rung) {
+  pdl_begin();
   using LY = NaiveLayout<D, MH>;
   constexpr int NG = D / VG;
   constexpr int CH = NaiveLanes<G>::CH;
@@ -628,14 +485,24 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     }
   }
   if (!ok) {
-    // let the copies still in flight land before the CTA exits
+    // let the copies still in flight land before the CTA exits, and leave empty
+    // partials (the status word already reports that the results are invalid)
     if (tid == 0) {
       const int hi = min(nblk - 1, k == 0 ? NST - 1 : k + NST - 2);
       for (int k2 = k; k2 <= hi; ++k2)
         mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
     }
-    naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, nb, hrow0, out, e_key, e_val, rung,
-                             reinterpret_cast<float*>(dsm), &S.last);
+    if (tid < G) {
+      for (int s2 = 0; s2 < (do_res ? 2 : 1); ++s2) {
+        const size_t pb = s2 ? ((size_t)unit * sc.max_chunks + nch) * G : pbase;
+        sc.part_s[(pb + tid) * 3 + 0] = -INFINITY;
+        sc.part_s[(pb + tid) * 3 + 1] = 0.f;
+        sc.part_s[(pb + tid) * 3 + 2] = 0.f;
+        sc.part_x[(pb + tid) * 3 + 0] = 0.f;
+        sc.part_x[(pb + tid) * 3 + 1] = -INFINITY;
+        sc.part_x[(pb + tid) * 3 + 2] = 0.f;
+      }
+    }
     return;
   }
   __syncthreads();  // every warp is past its last block: the stages are free
@@ -815,9 +682,129 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       sc.part_x[(rbase + tid) * 3 + 2] = mst[2 * tid + 1];
     }
   }
-  naive_arrive_merge<D, G>(sh, sc, nch + 1, nch, unit, nb, hrow0, out, e_key, e_val, rung,
-                           reinterpret_cast<float*>(dsm) + NaiveMergeAt<D, G>::AT, &S.last);
 }
+
+// Split-K combine of the streaming pass, one CTA per (batch row, query head),
+// launched as a programmatic dependent of the pass: it is scheduled while the
+// pass drains and waits (griddepcontrol.wait) until every CTA of the pass has
+// finished and its partials are visible.  Two rounds of independent loads: the
+// parts' statistics (max, sum, eta mass, largest Delta), then their output
+// vectors, spread over the CTA's warps and summed in shared memory.  Outputs
+// o / L, E_key from the largest Delta and the residual block's mass, and
+// E_val = eta mass / L.
+constexpr int CT = 512;         // combine threads: sixteen warps
+constexpr int CMAXP = 1024;     // most parts one unit may hold
+
+__device__ __forceinline__ float cblock_reduce(float v, bool is_max, float* sred) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, m);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  __syncthreads();  // sred may still be read by a previous reduction
+  if (lane == 0) sred[warp] = v;
+  __syncthreads();
+  float r = sred[0];
+  for (int w = 1; w < CT / 32; ++w) r = is_max ? fmaxf(r, sred[w]) : r + sred[w];
+  return r;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(CT) naive_combine_kernel(DecodeShape sh, Scratch sc, int grid_w,
+                                                            float* __restrict__ out,
+                                                            float* __restrict__ e_key,
+                                                            float* __restrict__ e_val,
+                                                            uint8_t* __restrict__ rung) {
+  constexpr int NWC = CT / 32;
+  constexpr int V4 = D / 4;          // float4 items of an output vector
+  constexpr int PPW = 32 / V4;       // parts per warp instruction
+  constexpr int SLOTS = NWC * PPW;   // parts in flight per round
+  constexpr int UNR = 4;
+  __shared__ float wts[CMAXP];
+  __shared__ float4 red[SLOTS][V4];
+  __shared__ float sred[NWC];
+  pdl_begin();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;  // b * Hq + h
+  const int b = row / sh.Hq, h = row - b * sh.Hq;
+  const int g = h / G, hh = h - g * G;
+  const int unit = b * sh.Hkv + g;
+  int nb, rr;
+  row_blocks(sh, b, nb, rr);
+  const int nch = min(grid_w, unit_ctas(sh.sms * NAIVE_CTAS_PER_SM, row_items(nb, rr),
+                                        sh.items_sum, naive_cap(nb, sc.max_chunks)));
+  const int nparts = nch + 1;  // the last part is the residual block's
+  const size_t base = (size_t)unit * sc.max_chunks * G + hh;  // partial index of part 0
+  // round 1: statistics
+  float M = -INFINITY, dA = 0.f;
+  for (int c = tid; c < nparts; c += CT) {
+    M = fmaxf(M, __ldcg(&sc.part_s[(base + (size_t)c * G) * 3]));
+    dA = fmaxf(dA, __ldcg(&sc.part_x[(base + (size_t)c * G) * 3]));
+  }
+  M = cblock_reduce(M, true, sred);
+  dA = cblock_reduce(dA, true, sred);
+  float ll = 0.f, el = 0.f;
+  for (int c = tid; c < nparts; c += CT) {
+    const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
+    const float m = __ldcg(ps);
+    const float w = m == -INFINITY ? 0.f : expf(m - M);
+    wts[c] = w;
+    ll = fmaf(__ldcg(ps + 1), w, ll);
+    el = fmaf(__ldcg(ps + 2), w, el);
+  }
+  const float L = cblock_reduce(ll, false, sred);
+  const float E = cblock_reduce(el, false, sred);  // its barrier also publishes wts
+  // round 2: output vectors, UNR parts per slot in flight
+  const int vi = lane % V4, sl = warp * PPW + lane / V4;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = sl; c0 < nparts; c0 += SLOTS * UNR) {
+    float4 v[UNR];
+    float wv[UNR];
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) {
+      const int c = c0 + i * SLOTS;
+      const bool in = c < nparts;
+      v[i] = in ? __ldcg(reinterpret_cast<const float4*>(sc.part_o + (base + (size_t)c * G) * D) + vi)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+      wv[i] = in ? wts[c] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) {
+      o.x = fmaf(v[i].x, wv[i], o.x);
+      o.y = fmaf(v[i].y, wv[i], o.y);
+      o.z = fmaf(v[i].z, wv[i], o.z);
+      o.w = fmaf(v[i].w, wv[i], o.w);
+    }
+  }
+  red[sl][vi] = o;
+  __syncthreads();
+  const size_t orow = (size_t)b * sh.Hq + h;
+  const float il = 1.f / L;
+  for (int i = tid; i < V4; i += CT) {
+    float4 s = red[0][i];
+    for (int k = 1; k < SLOTS; ++k) {
+      const float4 t = red[k][i];
+      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+    }
+    reinterpret_cast<float4*>(out + orow * D)[i] = make_float4(s.x * il, s.y * il, s.z * il, s.w * il);
+  }
+  if (tid == 0) {
+    // the residual part holds the residual block's own statistics
+    const float* px = sc.part_x + (base + (size_t)(nparts - 1) * G) * 3;
+    const float mr = __ldcg(px + 1);
+    const double mres = mr == -INFINITY ? 0.0 : (double)__ldcg(px + 2) * exp((double)mr - M) / L;
+    const float ek = nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
+    e_key[orow] = ek;
+    e_val[orow] = E / L;
+    rung[orow] = 0;
+    sc.ekey[orow] = ek;
+    sc.hflags[orow] = 0;
+    sc.kstar[orow] = 0;
+    sc.dense[orow] = 0;
+  }
+}
+
 
 // Grid width of the streaming pass: the most CTAs any unit receives.  Units
 // share sms * 4 CTAs (four resident per SM hold the whole grid, one wave, so a
@@ -841,16 +828,21 @@ cudaError_t naive_mh(const Tier1& t, const Strides& st, int unit0, const DecodeS
                      uint8_t* rung, int trace, cudaStream_t s) {
   const int nch = naive_chunks(sh, sc.max_chunks);
   const int smem = NST * NaiveLayout<D, MH>::STAGE;
-  // the merge keeps (nch + 1) * G weights, G inverse sums and NT float4 partial
-  // sums in the stage area, after what the CTAs still hold there
-  const size_t merge_floats =
-      (size_t)NaiveMergeAt<D, G>::AT + (size_t)(nch + 1) * G + G + 4 + (size_t)NT * 4;
-  if (merge_floats * 4 > (size_t)smem) return cudaErrorInvalidValue;
+  static_assert(NaiveScratchFloats<D, G>::N * 4 <= NST * NaiveLayout<D, false>::STAGE / 2,
+                "chunk-end scratch fits the stage area");
   cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G, MH>, (int)smem);
   if (e != cudaSuccess) return e;
-  naive_kernel<D, G, MH><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(
-      t, st, unit0, sh, q, sc, trace, out, e_key, e_val, rung);
-  return cudaGetLastError();
+  if (nch + 1 > CMAXP) return cudaErrorInvalidValue;
+  return launch_pdl(naive_kernel<D, G, MH>, dim3(nch, sh.B * sh.Hkv), dim3(NT), smem, s, t, st,
+                    unit0, sh, q, sc, trace, out, e_key, e_val, rung);
+}
+
+template <int D, int G>
+cudaError_t naive_combine_t(const DecodeShape& sh, const Scratch& sc, float* out, float* e_key,
+                            float* e_val, uint8_t* rung, cudaStream_t s) {
+  const int nch = naive_chunks(sh, sc.max_chunks);
+  return launch_pdl(naive_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(CT), 0, s, sh, sc, nch,
+                    out, e_key, e_val, rung);
 }
 
 template <int D, int G>
@@ -884,6 +876,27 @@ cudaError_t launch_naive(const Tier1& t, const Strides& st, int unit0, const Dec
     }
   }
 #undef CQA_NAIVE_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_naive_combine(const DecodeShape& sh, const Scratch& sc, float* out,
+                                 float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
+#define CQA_NC_CASE(DD, GG) return naive_combine_t<DD, GG>(sh, sc, out, e_key, e_val, rung, s)
+  if (sh.d == 128) {
+    switch (sh.G) {
+      case 1: CQA_NC_CASE(128, 1);
+      case 2: CQA_NC_CASE(128, 2);
+      case 4: CQA_NC_CASE(128, 4);
+      case 8: CQA_NC_CASE(128, 8);
+    }
+  } else {
+    switch (sh.G) {
+      case 1: CQA_NC_CASE(64, 1);
+      case 2: CQA_NC_CASE(64, 2);
+      case 4: CQA_NC_CASE(64, 4);
+    }
+  }
+#undef CQA_NC_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(THREADS) promote_kernel(Tier1 t, Strides st, i
                                                           Scratch sc,
                                                           const __half* __restrict__ kstage,
                                                           int stage_nb) {
+  pdl_begin();
   constexpr int LPR = D / 8;          // threads per token row, 8 channels each
   constexpr int RPC = THREADS / LPR;  // rows per pass
   constexpr int NPASS = BLK / RPC;
@@ -165,10 +166,11 @@ cudaError_t launch_promote_t(const Tier1& t, const Strides& st, int unit0, const
   dim3 grid(sh.nchunks, sh.B * sh.Hkv);
   if (!kstage) stage_nb = 0;
   if (mode == 0)
-    promote_kernel<D, G, 0><<<grid, THREADS, 0, s>>>(t, st, unit0, sh, q, sc, kstage, stage_nb);
+    return launch_pdl(promote_kernel<D, G, 0>, grid, dim3(THREADS), 0, s, t, st, unit0, sh, q, sc,
+                      kstage, stage_nb);
   else
-    promote_kernel<D, G, 1><<<grid, THREADS, 0, s>>>(t, st, unit0, sh, q, sc, kstage, stage_nb);
-  return cudaGetLastError();
+    return launch_pdl(promote_kernel<D, G, 1>, grid, dim3(THREADS), 0, s, t, st, unit0, sh, q, sc,
+                      kstage, stage_nb);
 }
 
 }  // namespace

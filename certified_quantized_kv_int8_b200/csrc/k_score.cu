@@ -110,6 +110,7 @@ template <int D, int G, bool MH>
 __global__ void __launch_bounds__(NT, 5)
     score_kernel(Tier1 t, Strides st, int unit0, DecodeShape sh, const __half* __restrict__ q,
                  Scratch sc) {
+  pdl_begin();
   using LY = ScoreLayout<D, MH>;
   constexpr int CPT = D / CH;     // lanes per token row
   constexpr int RPW = 32 / CPT;   // rows per warp instruction
@@ -401,8 +402,8 @@ cudaError_t launch_score_mh(const Tier1& t, const Strides& st, int unit0, const 
   const int smem = NST * ScoreLayout<D, MH>::STAGE;
   cudaError_t e = ensure_dynamic_smem((const void*)score_kernel<D, G, MH>, (int)smem);
   if (e != cudaSuccess) return e;
-  score_kernel<D, G, MH><<<dim3(nch, sh.B * sh.Hkv), NT, smem, s>>>(t, st, unit0, sh, q, sc);
-  return cudaGetLastError();
+  return launch_pdl(score_kernel<D, G, MH>, dim3(nch, sh.B * sh.Hkv), dim3(NT), smem, s, t, st,
+                    unit0, sh, q, sc);
 }
 
 template <int D, int G>

@@ -154,6 +154,7 @@ template <int G>
 __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, int unit0,
                                                          DecodeShape sh, cqa_thresholds th,
                                                          Scratch sc, int NP) {
+  pdl_begin();
   extern __shared__ __align__(16) unsigned char smem[];
   const int nbL = sh.nb_max;
   uint64_t* keys_all = reinterpret_cast<uint64_t*>(smem);
@@ -364,8 +365,8 @@ cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const 
   const size_t smem = (size_t)G * NP * 8 + (size_t)G * sh.nb_max * 4 + 2 * (size_t)sh.nb_max;
   cudaError_t e = ensure_dynamic_smem((const void*)select_kernel<G>, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<G><<<sh.B * sh.Hkv, THREADS, smem, s>>>(t, st, unit0, sh, th, sc, NP);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel<G>, dim3(sh.B * sh.Hkv), dim3(THREADS), smem, s, t, st, unit0, sh,
+                    th, sc, NP);
 }
 
 }  // namespace

@@ -283,9 +283,8 @@ enum {
   CQA_PHASE_DENSE_ATTEND = 9,  /* exact attention from Tier 2 (E_val post-check, reference) */
   CQA_PHASE_DENSE_COMBINE = 10,
   CQA_PHASE_PREFETCH = 11,     /* copy-engine copy of a layer's Tier-2 keys (not a kernel) */
-  CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1, whose
-                                  last CTA per (batch row, kv head) also combines */
-  CQA_PHASE_NAIVE_COMBINE = 13, /* reserved: no separate launch (the pass combines) */
+  CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1 */
+  CQA_PHASE_NAIVE_COMBINE = 13, /* certification off: split-K combine, outputs and bounds */
   CQA_PHASE_COUNT = 14
 };
 /* Start (or restart) profiling; max_launches bounds the recorded launches
