@@ -68,7 +68,6 @@ struct AttendSmem {
     float red[THREADS / LPR][D];
   } u;
   float m[G], l[G], e[G], alpha[G];
-  float eta_b;  // eta of the block being processed
 };
 
 // MODE 0: certified.  Logits come from scratch: INT8 for tail blocks, exact
@@ -147,16 +146,54 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
   }
 
   const uint8_t* bf = sc.bflags + ((size_t)b * sh.Hkv + g) * sh.nbm;
+  const float* etap = t.eta + u * st.eta;
   const int jstart = (chunk == 0 && rr > 0) ? -1 : j0;  // -1 = the residual block
+  // flags and eta_b of the next block are loaded one block ahead
+  auto blk_flags = [&](int j) -> uint8_t {
+    return (MODE == 0 && j >= 0 && j < j1) ? bf[j] : (uint8_t)(BF_KEY | BF_VAL);
+  };
+  auto blk_eta = [&](int j) -> float { return (MODE == 0 && j >= 0 && j < j1) ? etap[j] : 0.f; };
+  uint8_t fl_next = blk_flags(jstart);
+  float eta_next = blk_eta(jstart);
   for (int j = jstart; j < j1; ++j) {
     const bool resid = j < 0;
-    const uint8_t fl = (MODE == 0 && !resid) ? bf[j] : (uint8_t)(BF_KEY | BF_VAL);
+    const uint8_t fl = fl_next;
+    const float eta_b = eta_next;
+    fl_next = blk_flags(j + 1);
+    eta_next = blk_eta(j + 1);
     const bool vprom = resid || (fl & BF_VAL);
     const int ntok = resid ? rr : BLK;
     const size_t tok0 = resid ? (size_t)nb * BLK : (size_t)j * BLK;  // token index
+    const bool need_f16 = vprom || any_dense;
+    const bool need_i4 = MODE == 0 && !vprom && any_mixed;
+
+    // ---- this block's values, issued first: their latency overlaps the logits and softmax ----
+    uint4 vv[NPASS];
+    uint32_t wq[NPASS];
+    float2 mt[NPASS];
+#pragma unroll
+    for (int p = 0; p < NPASS; ++p) {
+      const int tt = p * RPC + row;
+      vv[p] = make_uint4(0u, 0u, 0u, 0u);
+      wq[p] = 0u;
+      mt[p] = make_float2(0.f, 0.f);
+      if (tt < ntok) {
+        if (need_f16) {
+          const __half* vsrc = resid ? t.vres + u * st.res + (size_t)tt * D
+                                     : t.v2 + u * st.tier2 + (tok0 + tt) * D;
+          vv[p] = *reinterpret_cast<const uint4*>(vsrc + cl * 8);
+        }
+        if (need_i4) {
+          wq[p] = *reinterpret_cast<const uint32_t*>(
+              t.vcodes + u * st.vcodes + ((size_t)j * BLK + tt) * (D / 2) + cl * 4);
+          const size_t mi = u * st.vmeta + (((size_t)j * BLK + tt) * NG + (cl * 8) / VG) * 2;
+          mt[p] = t.meta16 ? __half22float2(*reinterpret_cast<const __half2*>(t.vmeta_h + mi))
+                           : *reinterpret_cast<const float2*>(t.vmeta + mi);
+        }
+      }
+    }
 
     // ---- logits ----
-    if (MODE == 0 && tid == 0 && !resid) S.eta_b = t.eta[u * st.eta + j];  // overlaps the loads below
     if (MODE == 0) {
       const float* lp = sc.logits + hrow0 * sc.ls + tok0;
       for (int e = tid; e < G * BLK; e += THREADS) {
@@ -212,7 +249,7 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         S.l[h] = S.l[h] * alpha + lb;
         float ea = S.e[h] * alpha;
         const bool int4_here = MODE == 0 && !vprom && !sc.dense[hrow0 + h];
-        if (int4_here) ea += S.eta_b * lb;
+        if (int4_here) ea += eta_b * lb;
         S.e[h] = ea;
         S.m[h] = mnew;
         S.alpha[h] = alpha;
@@ -232,8 +269,6 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         acc[h][k].y *= al[h];
       }
     }
-    const bool need_f16 = vprom || any_dense;
-    const bool need_i4 = MODE == 0 && !vprom && any_mixed;
 #pragma unroll
     for (int p = 0; p < NPASS; ++p) {
       const int tt = p * RPC + row;
@@ -243,23 +278,12 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
       for (int h = 0; h < G; ++h) pw[h] = S.pp[h][tt];
       float2 vf[4];
       if (need_f16) {
-        const __half* vsrc = resid ? t.vres + u * st.res + (size_t)tt * D
-                                   : t.v2 + u * st.tier2 + (tok0 + tt) * D;
-        const uint4 vv = *reinterpret_cast<const uint4*>(vsrc + cl * 8);
-        const __half2* vh = reinterpret_cast<const __half2*>(&vv);
+        const __half2* vh = reinterpret_cast<const __half2*>(&vv[p]);
 #pragma unroll
         for (int k = 0; k < 4; ++k) vf[k] = __half22float2(vh[k]);
       }
       float2 cf[4];
-      float2 meta = make_float2(0.f, 0.f);
-      if (need_i4) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(
-            t.vcodes + u * st.vcodes + ((size_t)j * BLK + tt) * (D / 2) + cl * 4);
-        const size_t mi = u * st.vmeta + (((size_t)j * BLK + tt) * NG + (cl * 8) / VG) * 2;
-        meta = t.meta16 ? __half22float2(*reinterpret_cast<const __half2*>(t.vmeta_h + mi))
-                        : *reinterpret_cast<const float2*>(t.vmeta + mi);
-        u4x8_to_f2(w, cf);
-      }
+      if (need_i4) u4x8_to_f2(wq[p], cf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         if (vprom || dh[h]) {
@@ -267,8 +291,8 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
           for (int k = 0; k < 4; ++k)
             acc[h][k] = __ffma2_rn(make_float2(pw[h], pw[h]), vf[k], acc[h][k]);
         } else {
-          const float ws = pw[h] * meta.x;
-          zacc[h] = fmaf(pw[h], meta.y, zacc[h]);
+          const float ws = pw[h] * mt[p].x;
+          zacc[h] = fmaf(pw[h], mt[p].y, zacc[h]);
 #pragma unroll
           for (int k = 0; k < 4; ++k) acc[h][k] = __ffma2_rn(make_float2(ws, ws), cf[k], acc[h][k]);
         }

@@ -18,6 +18,7 @@
 // batch row) took rung 3 that way.  After the attention pass, a head whose
 // E_val exceeds eps_val also takes rung 3 (post-check, not counted for rung 4).
 #include "cqa_internal.cuh"
+#include "split_merge.cuh"
 
 namespace cqa {
 
@@ -202,102 +203,23 @@ __global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_threshol
   }
 }
 
-__device__ __forceinline__ float cwarp_max(float x) {
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
-  return x;
-}
-
-__device__ __forceinline__ float cwarp_sum(float x) {
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
-  return x;
-}
-
-// Merge the split-K partials of one head with a CTA of D threads: thread c
-// returns channel c of o / L; every thread gets L and E.
+// Outputs, E_val and the E_val post-check; one CTA of MERGE_THREADS threads per
+// (batch row, head).
 template <int D, int G>
-__device__ __forceinline__ float merge_head(const Scratch& sc, int nchunks, int unit, int hh,
-                                            float& L, float& E) {
-  constexpr int NW = D / 32;
-  __shared__ float wbuf[1024];
-  __shared__ float red[2][NW];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t base = (size_t)unit * sc.max_chunks * G + hh;  // partial index of chunk 0
-  float ml = -INFINITY;
-  for (int c = tid; c < nchunks; c += D) ml = fmaxf(ml, sc.part_s[(base + (size_t)c * G) * 3]);
-  ml = cwarp_max(ml);
-  if (lane == 0) red[0][warp] = ml;
-  __syncthreads();
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) M = fmaxf(M, red[0][w]);
-  __syncthreads();
-  float ll = 0.f, el = 0.f;
-  for (int c = tid; c < nchunks; c += D) {
-    const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
-    const float w = ps[0] == -INFINITY ? 0.f : expf(ps[0] - M);
-    if (c < 1024) wbuf[c] = w;
-    ll += ps[1] * w;
-    el += ps[2] * w;
-  }
-  ll = cwarp_sum(ll);
-  el = cwarp_sum(el);
-  if (lane == 0) {
-    red[0][warp] = ll;
-    red[1][warp] = el;
-  }
-  __syncthreads();
-  L = 0.f;
-  E = 0.f;
-#pragma unroll
-  for (int w = 0; w < NW; ++w) {
-    L += red[0][w];
-    E += red[1][w];
-  }
-  // o: batches of 16 independent loads so the chain of chunk partials does not
-  // serialise on memory latency
-  float o = 0.f;
-  for (int c0 = 0; c0 < nchunks; c0 += 16) {
-    float v[16], wv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = c0 + i;
-      v[i] = 0.f;
-      wv[i] = 0.f;
-      if (c < nchunks) {
-        const size_t pi = base + (size_t)c * G;
-        v[i] = sc.part_o[pi * D + tid];
-        if (c < 1024) {
-          wv[i] = wbuf[c];
-        } else {
-          const float mc = sc.part_s[pi * 3];
-          wv[i] = mc == -INFINITY ? 0.f : expf(mc - M);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o = fmaf(v[i], wv[i], o);
-  }
-  return o / L;
-}
-
-// Outputs, E_val and the E_val post-check; one CTA of D threads per (batch row, head).
-template <int D, int G>
-__global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
-                               float* __restrict__ out, float* __restrict__ e_key,
-                               float* __restrict__ e_val, uint8_t* __restrict__ rung) {
+__global__ void __launch_bounds__(MERGE_THREADS)
+    combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc, float* __restrict__ out,
+                   float* __restrict__ e_key, float* __restrict__ e_val,
+                   uint8_t* __restrict__ rung) {
   pdl_begin();
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   const int g = h / G, hh = h - g * G;
-  float L, E;
-  const float o = merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, L, E);
-  out[(size_t)row * D + threadIdx.x] = o;
+  const size_t base = ((size_t)b * sh.Hkv + g) * sc.max_chunks * G + hh;
+  const MergeStats ms = merge_parts<D, G>(sc, base, sh.nchunks, false, out + (size_t)row * D);
   if (threadIdx.x != 0) return;
   const uint8_t dv = sc.dense[row];
   uint8_t hf = sc.hflags[row];
-  const float ev = E / L;
+  const float ev = ms.E / ms.L;
   if (dv) {
     e_key[row] = 0.f;
     e_val[row] = 0.f;
@@ -317,20 +239,21 @@ __global__ void combine_kernel(DecodeShape sh, cqa_thresholds th, Scratch sc,
   sc.hflags[row] = hf;
 }
 
-// One CTA of D threads per (batch row, query head): heads recomputed by a
-// dense pass (all heads for cqa_dense_reference, DENSE_LATE heads otherwise).
+// One CTA of MERGE_THREADS threads per (batch row, query head): heads
+// recomputed by a dense pass (all heads for cqa_dense_reference, DENSE_LATE
+// heads otherwise).
 template <int D, int G>
-__global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
-                                     float* __restrict__ out, float* __restrict__ e_key,
-                                     float* __restrict__ e_val, uint8_t* __restrict__ rung) {
+__global__ void __launch_bounds__(MERGE_THREADS)
+    dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads, float* __restrict__ out,
+                         float* __restrict__ e_key, float* __restrict__ e_val,
+                         uint8_t* __restrict__ rung) {
   pdl_begin();
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   if (!all_heads && !(sc.dense[row] & DENSE_LATE)) return;
   const int g = h / G, hh = h - g * G;
-  float L, E;
-  const float o = merge_head<D, G>(sc, sh.nchunks, b * sh.Hkv + g, hh, L, E);
-  out[(size_t)row * D + threadIdx.x] = o;
+  const size_t base = ((size_t)b * sh.Hkv + g) * sc.max_chunks * G + hh;
+  merge_parts<D, G>(sc, base, sh.nchunks, false, out + (size_t)row * D);
   if (!all_heads && threadIdx.x == 0) {
     e_key[row] = 0.f;
     e_val[row] = 0.f;
@@ -341,14 +264,14 @@ __global__ void dense_combine_kernel(DecodeShape sh, Scratch sc, int all_heads,
 template <int D, int G>
 cudaError_t combine_t(const DecodeShape& sh, const cqa_thresholds& th, const Scratch& sc,
                       float* out, float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  return launch_pdl(combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(D), 0, s, sh, th, sc, out, e_key,
+  return launch_pdl(combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(MERGE_THREADS), 0, s, sh, th, sc, out, e_key,
                     e_val, rung);
 }
 
 template <int D, int G>
 cudaError_t dense_combine_t(const DecodeShape& sh, const Scratch& sc, int all_heads, float* out,
                             float* e_key, float* e_val, uint8_t* rung, cudaStream_t s) {
-  return launch_pdl(dense_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(D), 0, s, sh, sc,
+  return launch_pdl(dense_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(MERGE_THREADS), 0, s, sh, sc,
                     all_heads, out, e_key, e_val, rung);
 }
 

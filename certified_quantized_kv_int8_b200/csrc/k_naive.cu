@@ -44,6 +44,7 @@
 //     head) by the softmax lanes, which also accumulate the offset term.
 #include "bulk_pipe.cuh"
 #include "cqa_internal.cuh"
+#include "split_merge.cuh"
 
 namespace cqa {
 
@@ -687,45 +688,15 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
 // Split-K combine of the streaming pass, one CTA per (batch row, query head),
 // launched as a programmatic dependent of the pass: it is scheduled while the
 // pass drains and waits (griddepcontrol.wait) until every CTA of the pass has
-// finished and its partials are visible.  Two rounds of independent loads: the
-// parts' statistics (max, sum, eta mass, largest Delta), then their output
-// vectors, spread over the CTA's warps and summed in shared memory.  Outputs
-// o / L, E_key from the largest Delta and the residual block's mass, and
-// E_val = eta mass / L.
-constexpr int CT = 512;         // combine threads: sixteen warps
-constexpr int CMAXP = 1024;     // most parts one unit may hold
-
-__device__ __forceinline__ float cblock_reduce(float v, bool is_max, float* sred) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, m);
-    v = is_max ? fmaxf(v, o) : v + o;
-  }
-  __syncthreads();  // sred may still be read by a previous reduction
-  if (lane == 0) sred[warp] = v;
-  __syncthreads();
-  float r = sred[0];
-  for (int w = 1; w < CT / 32; ++w) r = is_max ? fmaxf(r, sred[w]) : r + sred[w];
-  return r;
-}
-
+// finished and its partials are visible.  The merge itself is merge_parts;
+// this kernel adds E_key from the largest Delta and the residual block's mass,
+// and E_val = eta mass / L.
 template <int D, int G>
-__global__ void __launch_bounds__(CT) naive_combine_kernel(DecodeShape sh, Scratch sc, int grid_w,
-                                                            float* __restrict__ out,
-                                                            float* __restrict__ e_key,
-                                                            float* __restrict__ e_val,
-                                                            uint8_t* __restrict__ rung) {
-  constexpr int NWC = CT / 32;
-  constexpr int V4 = D / 4;          // float4 items of an output vector
-  constexpr int PPW = 32 / V4;       // parts per warp instruction
-  constexpr int SLOTS = NWC * PPW;   // parts in flight per round
-  constexpr int UNR = 4;
-  __shared__ float wts[CMAXP];
-  __shared__ float4 red[SLOTS][V4];
-  __shared__ float sred[NWC];
+__global__ void __launch_bounds__(MERGE_THREADS)
+    naive_combine_kernel(DecodeShape sh, Scratch sc, int grid_w, float* __restrict__ out,
+                         float* __restrict__ e_key, float* __restrict__ e_val,
+                         uint8_t* __restrict__ rung) {
   pdl_begin();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / sh.Hq, h = row - b * sh.Hq;
   const int g = h / G, hh = h - g * G;
@@ -736,67 +707,16 @@ __global__ void __launch_bounds__(CT) naive_combine_kernel(DecodeShape sh, Scrat
                                         sh.items_sum, naive_cap(nb, sc.max_chunks)));
   const int nparts = nch + 1;  // the last part is the residual block's
   const size_t base = (size_t)unit * sc.max_chunks * G + hh;  // partial index of part 0
-  // round 1: statistics
-  float M = -INFINITY, dA = 0.f;
-  for (int c = tid; c < nparts; c += CT) {
-    M = fmaxf(M, __ldcg(&sc.part_s[(base + (size_t)c * G) * 3]));
-    dA = fmaxf(dA, __ldcg(&sc.part_x[(base + (size_t)c * G) * 3]));
-  }
-  M = cblock_reduce(M, true, sred);
-  dA = cblock_reduce(dA, true, sred);
-  float ll = 0.f, el = 0.f;
-  for (int c = tid; c < nparts; c += CT) {
-    const float* ps = sc.part_s + (base + (size_t)c * G) * 3;
-    const float m = __ldcg(ps);
-    const float w = m == -INFINITY ? 0.f : expf(m - M);
-    wts[c] = w;
-    ll = fmaf(__ldcg(ps + 1), w, ll);
-    el = fmaf(__ldcg(ps + 2), w, el);
-  }
-  const float L = cblock_reduce(ll, false, sred);
-  const float E = cblock_reduce(el, false, sred);  // its barrier also publishes wts
-  // round 2: output vectors, UNR parts per slot in flight
-  const int vi = lane % V4, sl = warp * PPW + lane / V4;
-  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = sl; c0 < nparts; c0 += SLOTS * UNR) {
-    float4 v[UNR];
-    float wv[UNR];
-#pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int c = c0 + i * SLOTS;
-      const bool in = c < nparts;
-      v[i] = in ? __ldcg(reinterpret_cast<const float4*>(sc.part_o + (base + (size_t)c * G) * D) + vi)
-                : make_float4(0.f, 0.f, 0.f, 0.f);
-      wv[i] = in ? wts[c] : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      o.x = fmaf(v[i].x, wv[i], o.x);
-      o.y = fmaf(v[i].y, wv[i], o.y);
-      o.z = fmaf(v[i].z, wv[i], o.z);
-      o.w = fmaf(v[i].w, wv[i], o.w);
-    }
-  }
-  red[sl][vi] = o;
-  __syncthreads();
   const size_t orow = (size_t)b * sh.Hq + h;
-  const float il = 1.f / L;
-  for (int i = tid; i < V4; i += CT) {
-    float4 s = red[0][i];
-    for (int k = 1; k < SLOTS; ++k) {
-      const float4 t = red[k][i];
-      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
-    }
-    reinterpret_cast<float4*>(out + orow * D)[i] = make_float4(s.x * il, s.y * il, s.z * il, s.w * il);
-  }
-  if (tid == 0) {
+  const MergeStats ms = merge_parts<D, G>(sc, base, nparts, true, out + orow * D);
+  if (threadIdx.x == 0) {
     // the residual part holds the residual block's own statistics
-    const float* px = sc.part_x + (base + (size_t)(nparts - 1) * G) * 3;
-    const float mr = __ldcg(px + 1);
-    const double mres = mr == -INFINITY ? 0.0 : (double)__ldcg(px + 2) * exp((double)mr - M) / L;
-    const float ek = nb > 0 ? (float)naive_e_key((double)dA, (double)dA, 1.0 - mres) : 0.f;
+    const float* pr = sc.part_x + (base + (size_t)(nparts - 1) * G) * 3;
+    const float mr = pr[1];
+    const double mres = mr == -INFINITY ? 0.0 : (double)pr[2] * exp((double)mr - ms.M) / ms.L;
+    const float ek = nb > 0 ? (float)naive_e_key((double)ms.XA, (double)ms.XA, 1.0 - mres) : 0.f;
     e_key[orow] = ek;
-    e_val[orow] = E / L;
+    e_val[orow] = ms.E / ms.L;
     rung[orow] = 0;
     sc.ekey[orow] = ek;
     sc.hflags[orow] = 0;
@@ -832,7 +752,6 @@ cudaError_t naive_mh(const Tier1& t, const Strides& st, int unit0, const DecodeS
                 "chunk-end scratch fits the stage area");
   cudaError_t e = ensure_dynamic_smem((const void*)naive_kernel<D, G, MH>, (int)smem);
   if (e != cudaSuccess) return e;
-  if (nch + 1 > CMAXP) return cudaErrorInvalidValue;
   return launch_pdl(naive_kernel<D, G, MH>, dim3(nch, sh.B * sh.Hkv), dim3(NT), smem, s, t, st,
                     unit0, sh, q, sc, trace, out, e_key, e_val, rung);
 }
@@ -841,7 +760,7 @@ template <int D, int G>
 cudaError_t naive_combine_t(const DecodeShape& sh, const Scratch& sc, float* out, float* e_key,
                             float* e_val, uint8_t* rung, cudaStream_t s) {
   const int nch = naive_chunks(sh, sc.max_chunks);
-  return launch_pdl(naive_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(CT), 0, s, sh, sc, nch,
+  return launch_pdl(naive_combine_kernel<D, G>, dim3(sh.B * sh.Hq), dim3(MERGE_THREADS), 0, s, sh, sc, nch,
                     out, e_key, e_val, rung);
 }
 

@@ -356,9 +356,244 @@ __global__ void __launch_bounds__(THREADS) select_kernel(Tier1 t, Strides st, in
   }
 }
 
+// Bitonic sort (ascending) of 32 * E keys by one warp, E keys per lane in
+// registers (lane l holds positions l*E .. l*E + E - 1 on exit): distances
+// below E are swaps inside a lane, the rest shuffles; no shared memory and no
+// barrier.
+template <int E>
+__device__ __forceinline__ void warp_sort(uint64_t (&v)[E], int lane) {
+  constexpr int n = 32 * E;
+#pragma unroll
+  for (int k = 2; k <= n; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          if ((r & j) == 0) {
+            const bool up = ((lane * E + r) & k) == 0;
+            const uint64_t a = v[r], b = v[r + j];
+            if ((a > b) == up) {
+              v[r] = b;
+              v[r + j] = a;
+            }
+          }
+        }
+      } else {
+        const int m = j / E;  // distance in lanes
+        const bool keep_min = ((lane & m) == 0) == (((lane * E) & k) == 0);
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[r], m);
+          v[r] = keep_min ? (o < v[r] ? o : v[r]) : (o > v[r] ? o : v[r]);
+        }
+      }
+    }
+  }
+}
+
+// The same selection for rows of at most 32 * E <= 256 sealed blocks (contexts
+// up to 16K tokens), where the 1024-thread kernel's named barriers set its
+// time: one warp per query head, the head's blocks in registers (E per lane),
+// its reductions, sort and K* scan done with shuffles; the CTA synchronises
+// only for the union P, the widening rounds and value promotion.  Same
+// quantities, same float64 scan, same tie order as select_kernel.
+template <int G, int E>
+__global__ void __launch_bounds__(32 * G) select_small_kernel(Tier1 t, Strides st, int unit0,
+                                                              DecodeShape sh, cqa_thresholds th,
+                                                              Scratch sc) {
+  pdl_begin();
+  constexpr int NP = 32 * E;
+  constexpr int NT = 32 * G;
+  __shared__ float mass_all[G][NP];
+  __shared__ uint8_t pflag[NP], vflag[NP];
+  __shared__ int kst[G], kold[G];
+  __shared__ double ekey_s[G];
+  __shared__ int any_fail;
+  __shared__ int npro_s;
+  __shared__ unsigned hf_s[G];
+
+  const int unit = blockIdx.x;
+  const int b = unit / sh.Hkv, g = unit - b * sh.Hkv;
+  const size_t u = (size_t)unit0 + unit;
+  const size_t hrow0 = (size_t)b * sh.Hq + (size_t)g * G;
+  const int tid = threadIdx.x, h = tid >> 5, lane = tid & 31;
+  const bool naive = th.naive != 0;
+  int nb, r_unused;  // this row's sealed blocks (at most NP)
+  row_blocks(sh, b, nb, r_unused);
+  const float* e8 = sc.ell8 + (hrow0 + h) * sh.nbm;
+  const float* dl = sc.delta + (hrow0 + h) * sh.nbm;
+
+  for (int j = tid; j < NP; j += NT) {
+    pflag[j] = 0;
+    vflag[j] = 0;
+  }
+  if (tid < G) hf_s[tid] = 0;
+  if (tid == 0) npro_s = 0;
+
+  // ---- per head: log-sum-exp, masses, Delta max; lane holds blocks lane + 32 i ----
+  const float eres = sc.ell_res[hrow0 + h];
+  float ev[E], dv[E], ms[E];
+  float mx = eres, dmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const int j = lane + 32 * i;
+    ev[i] = j < nb ? e8[j] : -INFINITY;
+    dv[i] = j < nb ? dl[j] : 0.f;
+    mx = fmaxf(mx, ev[i]);
+    dmax = fmaxf(dmax, dv[i]);
+  }
+  mx = wmax(mx);
+  const float dA = wmax(dmax);
+  double ssum = 0.0;
+#pragma unroll
+  for (int i = 0; i < E; ++i)
+    if (lane + 32 * i < nb) ssum += (double)expf(ev[i] - mx);
+  if (lane == 0 && eres > -INFINITY) ssum += (double)expf(eres - mx);
+  ssum = wsum(ssum);
+  const float lse = mx + (float)log(ssum);
+  uint64_t v[E];  // sort keys; any starting arrangement sorts to the same order
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const int j = lane + 32 * i;
+    ms[i] = j < nb ? expf(ev[i] - lse) : 0.f;
+    mass_all[h][j] = ms[i];
+    v[i] = j < nb ? sort_key(ev[i], (uint32_t)j) : ~0ull;
+  }
+  const float m_res_f = eres > -INFINITY ? expf(eres - lse) : 0.f;
+  warp_sort<E>(v, lane);  // now position lane * E + r
+  __syncwarp();           // the head's masses are in shared memory
+
+  // ---- K*: float64 inclusive scan of the sorted masses ----
+  int kstar = 0;
+  if (naive) {
+    kstar = 0;
+  } else if (th.tau_cov >= 1.0f) {
+    kstar = nb;
+  } else {
+    const double tau = (double)th.tau_cov;
+    const double m_res = (double)m_res_f;
+    double mr[E], local = 0.0;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int p = lane * E + r;
+      mr[r] = p < nb ? (double)mass_all[h][(int)(v[r] & 0xffffffffu)] : 0.0;
+      local += mr[r];
+    }
+    double incl = local;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, m);
+      if (lane >= m) incl += y;
+    }
+    double run = m_res + (incl - local);
+    int cnt = 0;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      if (lane * E + r < nb) {
+        run += mr[r];
+        cnt += run < tau ? 1 : 0;  // prefix of position + 1 blocks below tau
+      }
+    }
+    cnt = wsum(cnt);
+    kstar = (m_res < tau) ? min(nb, cnt + 1) : 0;
+  }
+  if (lane == 0) kst[h] = kstar;
+#pragma unroll
+  for (int r = 0; r < E; ++r)
+    if (lane * E + r < kstar) pflag[(int)(v[r] & 0xffffffffu)] = 1;
+  __syncthreads();
+
+  // ---- E_key and rung-1 widening ----
+  for (int round = 0;; ++round) {
+    float dT = 0.f;
+    double m8T = 0.0;
+    int ntail = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const int j = lane + 32 * i;
+      if (j < nb && !pflag[j]) {
+        dT = fmaxf(dT, dv[i]);
+        m8T += (double)ms[i];
+        ++ntail;
+      }
+    }
+    dT = wmax(dT);
+    m8T = wsum(m8T);
+    ntail = wsum(ntail);
+    if (lane == 0) ekey_s[h] = ntail ? e_key_bound((double)dT, (double)dA, m8T) : 0.0;
+    __syncthreads();
+    if (tid == 0) {
+      any_fail = 0;
+      for (int hh = 0; hh < G; ++hh) {
+        kold[hh] = kst[hh];
+        if (!naive && ekey_s[hh] > (double)th.eps_key && round < th.max_expand) {
+          kst[hh] = min(nb, max(1, 2 * kst[hh]));
+          hf_s[hh] |= HF_WIDENED;
+          any_fail = 1;
+        }
+      }
+    }
+    __syncthreads();
+    if (!any_fail) break;
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int p = lane * E + r;
+      if (p >= kold[h] && p < kst[h]) pflag[(int)(v[r] & 0xffffffffu)] = 1;
+    }
+    __syncthreads();
+  }
+
+  // ---- rung 2: value promotion ----
+  const float* eta = t.eta + u * st.eta;
+  if (!naive) {
+    for (int j = tid; j < nb; j += NT) {
+      const float e = eta[j];
+      uint8_t vp = 0;
+      for (int hh = 0; hh < G; ++hh) {
+        if (mass_all[hh][j] * e > th.v_tol) {
+          vp = 1;
+          atomicOr(&hf_s[hh], (unsigned)HF_VALUE);
+        }
+      }
+      vflag[j] = vp;
+    }
+  }
+  __syncthreads();
+
+  uint8_t* bf = sc.bflags + ((size_t)b * sh.Hkv + g) * sh.nbm;
+  int npro = 0;
+  for (int j = tid; j < nb; j += NT) {
+    bf[j] = (pflag[j] ? BF_KEY : 0) | (vflag[j] ? BF_VAL : 0);
+    npro += pflag[j] ? 1 : 0;
+  }
+  npro = wsum(npro);
+  if (lane == 0 && npro) atomicAdd(&npro_s, npro);
+  __syncthreads();
+  if (tid == 0 && sc.promo) sc.promo[u] = npro_s;
+  if (tid < G) {
+    const int hh = tid;
+    unsigned f = hf_s[hh];
+    if (!naive && ekey_s[hh] > (double)th.eps_key) f |= HF_KEYFAIL;
+    sc.hflags[hrow0 + hh] = (uint8_t)f;
+    sc.kstar[hrow0 + hh] = kst[hh];
+    sc.ekey[hrow0 + hh] = (float)ekey_s[hh];
+  }
+}
+
 template <int G>
 cudaError_t launch_select_t(const Tier1& t, const Strides& st, int unit0, const DecodeShape& sh,
                             const cqa_thresholds& th, const Scratch& sc, cudaStream_t s) {
+  if (sh.nb_max <= 256) {  // one warp per head, keys in registers
+    const dim3 grid(sh.B * sh.Hkv), block(32 * G);
+    if (sh.nb_max <= 32)
+      return launch_pdl(select_small_kernel<G, 1>, grid, block, 0, s, t, st, unit0, sh, th, sc);
+    if (sh.nb_max <= 64)
+      return launch_pdl(select_small_kernel<G, 2>, grid, block, 0, s, t, st, unit0, sh, th, sc);
+    if (sh.nb_max <= 128)
+      return launch_pdl(select_small_kernel<G, 4>, grid, block, 0, s, t, st, unit0, sh, th, sc);
+    return launch_pdl(select_small_kernel<G, 8>, grid, block, 0, s, t, st, unit0, sh, th, sc);
+  }
   int NP = 2;
   while (NP < sh.nb_max) NP <<= 1;
   if (NP < THREADS / G) NP = THREADS / G;  // at least one key per thread of a head group

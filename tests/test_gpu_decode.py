@@ -87,6 +87,29 @@ def test_decode_fp16_meta(cqa, name, ctx, naive):
     assert len(log.entries) <= 2
 
 
+@pytest.mark.parametrize("nb", [40, 200, 256, 257])
+@pytest.mark.parametrize("case", ["default", "widen", "tau0.9_vtol", "naive"])
+def test_decode_selection_sizes(cqa, nb, case):
+    """Coverage selection runs one warp per query head with the head's blocks in
+    registers up to 256 sealed blocks (32, 64, 128 or 256 sort keys per head),
+    and the 1024-thread kernel above that: rows on both sides of each size, with
+    widening, a tail with value promotion, and certification off."""
+    w = sk.WORKLOADS["tiny"]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), **TINY_TH[case]})
+    log = _check(cqa, w, nb * 64 + 17, th, label=f"nb{nb} {case}")
+    assert len(log.entries) <= 1
+
+
+@pytest.mark.parametrize("nb", [200, 300])
+def test_decode_selection_sizes_g4(cqa, nb):
+    """The same two selection kernels at head_dim 128 with four query heads per kv
+    head (eight kv heads, a tail and value promotion)."""
+    w = sk.WORKLOADS["llama8b_8k_1layer"]
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.9, "v_tol": 2e-3})
+    log = _check(cqa, w, nb * 64 + 9, th, label=f"g4 nb{nb}")
+    assert len(log.entries) <= 2
+
+
 def test_decode_llama8b_8k(cqa):
     w = sk.WORKLOADS["llama8b_8k_1layer"]
     th = cqa.Thresholds(**sk.default_thresholds(w))
