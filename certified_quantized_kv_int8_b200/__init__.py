@@ -48,7 +48,7 @@ EXPORTED_SYMBOLS = (
 
 PHASES = ("append_seal", "append_tail", "score", "select", "promote", "decide", "dense_keys",
           "attend", "combine", "dense_attend", "dense_combine", "prefetch", "naive",
-          "naive_combine")
+          "naive_combine", "promote_staged")
 
 
 class _Config(ctypes.Structure):

@@ -673,7 +673,7 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
   const __half* kstage = slot >= 0 ? cc->kstage[slot] : nullptr;
   const int stage_nb = slot >= 0 ? cc->stage_nb[slot] : 0;
   if (naive) {
-    // certification off: one streaming pass over Tier 1 (its last CTA per unit combines)
+    // certification off: one streaming pass over Tier 1, then the split-K combine
     cudaError_t e = run_phase(cc, CQA_PHASE_NAIVE, s, 1, [&] {
       return launch_naive(cc->t, cc->st, unit0, sh, qh, cc->sc, out, e_key, e_val, rung,
                           trace != nullptr, s);
@@ -692,10 +692,12 @@ int cqa_decode(cqa_cache* cc, int layer, const void* q, const cqa_thresholds* th
     e = run_phase(cc, CQA_PHASE_SELECT, s, 1,
                   [&] { return launch_select(cc->t, cc->st, unit0, sh, tv, cc->sc, s); });
   if (e == cudaSuccess && slot >= 0) e = cudaStreamWaitEvent(s, cc->ev_ready[slot], 0);
-  if (e == cudaSuccess && !naive && sh.nb_max > 0)
+  if (e == cudaSuccess && !naive && sh.nb_max > 0) {
     e = run_phase(cc, CQA_PHASE_PROMOTE, s, 1, [&] {
       return launch_promote(cc->t, cc->st, unit0, sh, qh, cc->sc, 0, kstage, stage_nb, s);
     });
+    if (cc->prof_on && kstage) cc->prof_launches[CQA_PHASE_PROMOTE_STAGED] += 1;
+  }
   if (e == cudaSuccess)
     e = run_phase(cc, CQA_PHASE_DECIDE, s, 1,
                   [&] { return launch_decide(sh, tv, need_dense, cc->sc, s); });

@@ -33,15 +33,13 @@ struct KI {
 __device__ __forceinline__ bool before(KI a, KI b) { return a.k > b.k || (a.k == b.k && a.i < b.i); }
 
 // Rank check and the rung 3 / rung 4 decision, before the attention pass.
-// One CTA of DT threads per (batch row, query head).  The head's INT8 and FP16
-// block log-masses and the block flags are staged in shared memory when they
-// fit (else read in place).  The two top-r lists are built one rank at a time
-// by CTA-wide arg-bests under the (key desc, index asc) orders; their union U
-// (at most 2 * MAX_RANK_R blocks) is then compared pair by pair, one pair per
-// thread per round.  The last CTA of a batch row to finish takes the
+// One warp per (batch row, query head), DWH heads per CTA; no CTA barrier.
+// The two top-r lists are built one rank at a time by warp-wide arg-bests
+// under the (key desc, index asc) orders, over the head's promoted blocks held
+// in registers (E per lane: rows of at most 32 * E <= 256 blocks); their union
+// U (at most 2 * MAX_RANK_R blocks) is then compared pair by pair.  The last head of a batch row to finish takes the
 // whole-layer decision (rung 4).
-constexpr int DT = 256;
-constexpr int DW = DT / 32;
+constexpr int DWH = 8;  // heads (warps) per CTA
 
 __device__ __forceinline__ KI ki_best(KI a, KI b) { return before(b, a) ? b : a; }
 
@@ -56,7 +54,135 @@ __device__ __forceinline__ KI warp_best(KI v) {
   return v;
 }
 
-__global__ void __launch_bounds__(DT) decide_kernel(DecodeShape sh, cqa_thresholds th,
+template <int E>
+__global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_thresholds th,
+                                                          int need_dense, Scratch sc) {
+  pdl_begin();
+  __shared__ int top8[DWH][MAX_RANK_R], top16[DWH][MAX_RANK_R];
+  __shared__ int uni[DWH][2 * MAX_RANK_R];
+  __shared__ float u8[DWH][2 * MAX_RANK_R], u16[DWH][2 * MAX_RANK_R];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row_i = blockIdx.x * DWH + w;  // b * Hq + h
+  if (row_i >= sh.B * sh.Hq) return;       // the whole warp: nothing below waits on it
+  const int b = row_i / sh.Hq, h = row_i - b * sh.Hq;
+  const int unit = b * sh.Hkv + h / sh.G;
+  const size_t row = (size_t)row_i;
+  int nb, r_unused;  // this batch row's sealed blocks
+  row_blocks(sh, b, nb, r_unused);
+  const uint8_t* bf = sc.bflags + (size_t)unit * sh.nbm;
+  const float* e8 = sc.ell8 + row * sh.nbm;
+  const float* e16 = sc.ell16 + row * sh.nbm;
+  static_assert(E >= 1 && E <= 8, "rows of at most 256 blocks");
+  float k8[E], k16[E];
+  bool pr[E];
+  int np = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const int j = lane + 32 * i;
+    pr[i] = j < nb && (bf[j] & BF_KEY);
+    k8[i] = pr[i] ? e8[j] : 0.f;
+    k16[i] = pr[i] ? e16[j] : 0.f;
+    np += pr[i] ? 1 : 0;
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) np += __shfl_xor_sync(0xffffffffu, np, m);
+  const int r = min(min(th.rank_r, MAX_RANK_R), np);
+  // the two top-r lists
+  KI p8{INFINITY, -1}, p16{INFINITY, -1};
+  for (int k = 0; k < r; ++k) {
+    KI c8{-INFINITY, 0x7fffffff}, c16{-INFINITY, 0x7fffffff};
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      if (!pr[i]) continue;
+      const KI a{k8[i], lane + 32 * i}, a2{k16[i], lane + 32 * i};
+      if (before(p8, a) && before(a, c8)) c8 = a;
+      if (before(p16, a2) && before(a2, c16)) c16 = a2;
+    }
+    p8 = warp_best(c8);
+    p16 = warp_best(c16);
+    if (lane == 0) {
+      top8[w][k] = p8.i;
+      top16[w][k] = p16.i;
+    }
+  }
+  __syncwarp();
+  // union: the INT8 list, then the FP16 entries it does not hold
+  int base = r;
+  for (int k0 = 0; k0 < r; k0 += 32) {
+    const int k = k0 + lane;
+    bool fresh = false;
+    if (k < r) {
+      fresh = true;
+      for (int i = 0; i < r; ++i) fresh &= top8[w][i] != top16[w][k];
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, fresh);
+    if (fresh) uni[w][base + __popc(m & ((1u << lane) - 1u))] = top16[w][k];
+    base += __popc(m);
+  }
+  for (int k = lane; k < r; k += 32) uni[w][k] = top8[w][k];
+  const int nu = base;
+  __syncwarp();
+  for (int k = lane; k < nu; k += 32) {
+    const int a = uni[w][k];
+    u8[w][k] = e8[a];
+    u16[w][k] = e16[a];
+  }
+  __syncwarp();
+  // discordant pairs of U: the two orders place the pair the other way round
+  int disc = 0;
+  for (int pi = lane; pi < nu * nu; pi += 32) {
+    const int i = pi / nu, j = pi - i * nu;
+    if (i >= j) continue;
+    const int a = uni[w][i], c = uni[w][j];
+    const bool a8 = before(KI{u8[w][i], a}, KI{u8[w][j], c});
+    const bool a16 = before(KI{u16[w][i], a}, KI{u16[w][j], c});
+    disc += a8 != a16 ? 1 : 0;
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) disc += __shfl_xor_sync(0xffffffffu, disc, m);
+  const bool fail = disc > th.rank_tol;
+  const bool naive = th.naive != 0;
+  int last = 0;
+  if (lane == 0) {
+    uint8_t hf = sc.hflags[row];
+    if (!naive && fail) hf |= HF_RANKFAIL;
+    sc.hflags[row] = hf;
+    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
+    if (is3) atomicAdd(&sc.dcnt[2 * b], 1);
+    __threadfence();
+    last = atomicAdd(&sc.dcnt[2 * b + 1], 1) == sh.Hq - 1;
+  }
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
+  // the last head of the batch row: rung 3 per head, or rung 4 for the layer
+  __threadfence();
+  int n3 = 0;
+  if (lane == 0) n3 = atomicAdd(&sc.dcnt[2 * b], 0);
+  n3 = __shfl_sync(0xffffffffu, n3, 0);
+  const bool layer = !naive && n3 >= need_dense;
+  for (int hh = lane; hh < sh.Hq; hh += 32) {
+    const size_t rw = (size_t)b * sh.Hq + hh;
+    const uint8_t hf = __ldcg(&sc.hflags[rw]);
+    const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
+    sc.dense[rw] = layer ? 4 : (is3 ? 3 : 0);
+  }
+  if (lane == 0) {
+    sc.dcnt[2 * b] = 0;
+    sc.dcnt[2 * b + 1] = 0;
+  }
+}
+
+// The same decision for rows of more than 256 blocks: one CTA of DT threads per
+// (batch row, query head).  The head's INT8 and FP16
+// block log-masses and the block flags are staged in shared memory when they
+// fit (else read in place).  The two top-r lists are built one rank at a time
+// by CTA-wide arg-bests under the (key desc, index asc) orders; their union U
+// (at most 2 * MAX_RANK_R blocks) is then compared pair by pair, one pair per
+// thread per round.  The last CTA of a batch row to finish takes the
+// whole-layer decision (rung 4).
+constexpr int DT = 256;
+constexpr int DW = DT / 32;
+
+__global__ void __launch_bounds__(DT) decide_cta_kernel(DecodeShape sh, cqa_thresholds th,
                                                     int need_dense, Scratch sc, int staged) {
   pdl_begin();
   extern __shared__ __align__(16) unsigned char dsm[];
@@ -304,16 +430,26 @@ cudaError_t launch_combine(const DecodeShape& sh, const cqa_thresholds& th, cons
 
 cudaError_t launch_decide(const DecodeShape& sh, const cqa_thresholds& th, int need_dense,
                           const Scratch& sc, cudaStream_t s) {
-  // stage the head's keys and flags in shared memory up to 96 KiB
+  const dim3 grid((sh.B * sh.Hq + DWH - 1) / DWH), block(32 * DWH);
+  if (sh.nb_max <= 32)
+    return launch_pdl(decide_kernel<1>, grid, block, 0, s, sh, th, need_dense, sc);
+  if (sh.nb_max <= 64)
+    return launch_pdl(decide_kernel<2>, grid, block, 0, s, sh, th, need_dense, sc);
+  if (sh.nb_max <= 128)
+    return launch_pdl(decide_kernel<4>, grid, block, 0, s, sh, th, need_dense, sc);
+  if (sh.nb_max <= 256)
+    return launch_pdl(decide_kernel<8>, grid, block, 0, s, sh, th, need_dense, sc);
+  // longer rows: a CTA per head, the head's keys and flags staged in shared
+  // memory up to 96 KiB
   const size_t bytes = (size_t)sh.nb_max * 9;
   const int staged = bytes <= 96u * 1024u ? 1 : 0;
   const int smem = staged ? (int)((bytes + 15) / 16 * 16) : 0;
   if (smem > 48 * 1024) {
-    cudaError_t e = ensure_dynamic_smem((const void*)decide_kernel, smem);
+    cudaError_t e = ensure_dynamic_smem((const void*)decide_cta_kernel, smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(decide_kernel, dim3(sh.B * sh.Hq), dim3(DT), smem, s, sh, th, need_dense, sc,
-                    staged);
+  return launch_pdl(decide_cta_kernel, dim3(sh.B * sh.Hq), dim3(DT), smem, s, sh, th, need_dense,
+                    sc, staged);
 }
 
 cudaError_t launch_dense_combine(const DecodeShape& sh, const Scratch& sc, int all_heads,

@@ -285,7 +285,10 @@ enum {
   CQA_PHASE_PREFETCH = 11,     /* copy-engine copy of a layer's Tier-2 keys (not a kernel) */
   CQA_PHASE_NAIVE = 12,        /* certification off: one streaming pass over Tier 1 */
   CQA_PHASE_NAIVE_COMBINE = 13, /* certification off: split-K combine, outputs and bounds */
-  CQA_PHASE_COUNT = 14
+  CQA_PHASE_PROMOTE_STAGED = 14, /* count only, never timed: the CQA_PHASE_PROMOTE launches
+                                  * that read the keys from a device copy staged by the
+                                  * prefetch instead of from Tier 2 over the host link */
+  CQA_PHASE_COUNT = 15
 };
 /* Start (or restart) profiling; max_launches bounds the recorded launches
  * (further launches are counted but not timed). */
