@@ -199,14 +199,21 @@ def traffic_record(kernel: str):
     return rec
 
 
-def decision_census(cache, qs, th, w, device) -> dict:
-    """Decode every layer once more with a trace and count the decisions."""
+TIE_REL = 1e-6  # relative band of a threshold tie
+
+
+def decision_census(cache, qs_steps, th, w, device) -> dict:
+    """Decode every layer once more with a trace, for the queries of each step in
+    qs_steps (a list of per-layer query lists), and count the decisions; counts are
+    summed over all those decodes (c["decodes"] of them)."""
     L, B, Hkv, G = w.n_layers, w.batch, w.n_kv_heads, w.group
     c = dict(blocks=0, key_promoted=0, value_promoted=0, heads=0, rungs=[0] * 5, units=0,
              dense_units=0, dense_unit_blocks=0, dense_unit_nonpromoted=0,
-             vp_or_dense_blocks=0, int4_blocks=0, blocks_per_layer=0, rank_fail=0, key_fail=0)
+             vp_or_dense_blocks=0, int4_blocks=0, blocks_per_layer=0, rank_fail=0, key_fail=0,
+             decodes=0, ties=dict(coverage=0, e_key=0, value_promotion=0))
     e_key, e_val = [], []
-    for layer in range(L):
+    for qs, layer in ((qs, layer) for qs in qs_steps for layer in range(L)):
+        c["decodes"] += 1
         tr = cache.alloc_trace(layer)
         o = cache.alloc_outputs()
         cache.decode(layer, qs[layer], th, outputs=o, trace=tr)
@@ -240,6 +247,32 @@ def decision_census(cache, qs, th, w, device) -> dict:
         cert = rg < 3  # dense heads report 0 for both bounds
         e_key.append(o[1].cpu().numpy()[cert])
         e_val.append(o[2].cpu().numpy()[cert])
+        # decisions that sat within TIE_REL of their threshold (float32 rounding
+        # could have taken either side): the coverage sum at some rank, E_key, and
+        # a block's estimated value contribution
+        ek_all = o[1].cpu().numpy()
+        c["ties"]["e_key"] += int((cert & (np.abs(ek_all - th.eps_key)
+                                           <= TIE_REL * abs(th.eps_key))).sum())
+        e8 = tr["ell8"].cpu().numpy()
+        eres = tr["ell_res"].cpu().numpy()
+        eta = cache.export(layer, 4)  # EXPORT_ETA: [B][Hkv][nb], or per-row arrays
+        for b in range(B):
+            n = int(nb_row[b])
+            if n == 0:
+                continue
+            x = e8[b, :, :n].astype(np.float64)  # [Hq][n]
+            mx = np.maximum(x.max(axis=1), eres[b])
+            tot = np.exp(x - mx[:, None]).sum(axis=1) + np.where(
+                np.isfinite(eres[b]), np.exp(eres[b] - mx), 0.0)
+            m8 = np.exp(x - mx[:, None]) / tot[:, None]
+            mres = np.where(np.isfinite(eres[b]), np.exp(eres[b] - mx), 0.0) / tot
+            cum = mres[:, None] + np.cumsum(-np.sort(-m8, axis=1), axis=1)
+            near = np.abs(cum - th.tau_cov) <= TIE_REL * th.tau_cov
+            c["ties"]["coverage"] += int((near.any(axis=1) & (rg[b] < 3)).sum())
+            eb = np.asarray(eta[b] if isinstance(eta, list) else eta[b])[:, :n]  # [Hkv][n]
+            contrib = m8.reshape(Hkv, G, n) * eb[:, None, :]
+            c["ties"]["value_promotion"] += int(
+                (np.abs(contrib - th.v_tol) <= TIE_REL * th.v_tol).any(axis=1).sum())
     ek, ev = np.concatenate(e_key), np.concatenate(e_val)
     pct = (50, 90, 99, 100)
     c["e_key_pct"] = {f"p{q}": float(np.percentile(ek, q)) for q in pct} if ek.size else None
@@ -251,9 +284,9 @@ def phase_bytes(c: dict, w: sk.Workload, staged_frac: float = 0.0) -> dict:
     """Algorithmic bytes per launch of each decode phase: (host link, HBM).
     staged_frac: share of promote launches whose keys came from the device copy
     made by the whole-layer key prefetch (read from HBM instead of Tier 2)."""
-    L, d, G = w.n_layers, w.head_dim, w.group
+    d, G = w.head_dim, w.group
     kblk = BLOCK * d * 2  # FP16 keys (or values) of one block and kv head
-    per = lambda x: x / L  # noqa: E731  (census counts are over all layers)
+    per = lambda x: x / c["decodes"]  # noqa: E731  (census counts are over all its decodes)
     nblk = per(c["blocks"])
     kp = per(c["key_promoted"]) * kblk
     return {
@@ -311,7 +344,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     n_naive = args.steps
     # headline loops run without per-kernel events; a second, profiled pass of
     # each supplies the per-kernel times (events between kernels add gaps)
-    total_steps = args.warmup + 2 * args.steps + n_e2e + 2 * n_naive
+    total_steps = args.warmup + 2 * args.steps + n_e2e + args.warmup + 2 * n_naive
     max_ctx = w.ctx + (total_steps if appends else 0)
     wr = dataclasses.replace(w, seed=w.seed + rank)  # independent replica per rank
 
@@ -346,6 +379,12 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     inputs = [step_inputs(s) for s in range(total_steps)]
     outs = cache.alloc_outputs()
     stream = torch.cuda.current_stream(device)
+    # Tier 1 of a whole step below twice the L2: flush the L2 between steps
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    step_t1 = sum(n // BLOCK for layer in range(L) for n in lens0) * Hkv * \
+        tier1_bytes_per_block(d, args.meta_fp16)
+    flush = (torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device)
+             if step_t1 < 2 * l2_bytes else None)
 
     # the timed loops call the C entry points with marshalled arguments prepared
     # once, so the host enqueues a layer in a few microseconds (the e2e pass below
@@ -378,19 +417,33 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     def timed(first, n, thr, profile=False, label="timed"):
         barrier(dist, device)
         torch.cuda.synchronize(device)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if profile:
             cache.profile_begin(1 << 20)
         torch.cuda.nvtx.range_push(label)  # lets a profiler select the timed steps
-        a.record(stream)
-        for s in range(first, first + n):
-            run_step(s, thr)
-        b.record(stream)
+        if flush is None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for s in range(first, first + n):
+                run_step(s, thr)
+            b.record(stream)
+            evs = [(a, b)]
+        else:
+            # a step whose data fits in L2: the L2 is flushed before each step,
+            # outside that step's events (the flush also keeps the GPU busy
+            # while the host enqueues the step)
+            evs = []
+            for s in range(first, first + n):
+                flush.fill_(s & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                run_step(s, thr)
+                b.record(stream)
+                evs.append((a, b))
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(device)
         prof = cache.profile_end() if profile else None
         barrier(dist, device)
-        return a.elapsed_time(b) * 1e-3, prof
+        return sum(a.elapsed_time(b) for a, b in evs) * 1e-3, prof
 
     for s in range(args.warmup):
         run_step(s, th)
@@ -408,7 +461,12 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     phase_ms, phase_n, untimed = prof
 
     # census of the decisions (untimed, on the state after the timed steps)
-    census = decision_census(cache, inputs[args.warmup + args.steps - 1][0], th, w, device)
+    # (several steps' queries when a step has few layers, so that one step's
+    # decisions do not stand for all of them)
+    n_census = max(1, min(16, 64 // L))
+    census = decision_census(
+        cache, [inputs[args.warmup + args.steps - 1 - k][0] for k in range(n_census)], th, w,
+        device)
 
     # every layer once more with no copy in flight: in the step, the key
     # prefetch's host-to-device copy delays each kernel launch by about 20 us,
@@ -441,9 +499,19 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         d2h = L * sum(t.numel() * t.element_size() for t in outs)
         barrier(dist, device)
         torch.cuda.synchronize(device)
+        # one pair of events around all steps (host gaps between steps included);
+        # with an L2 flush, one pair per step with the flush between them
+        evs = []
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(n_e2e):
+            if flush is not None:
+                if i:
+                    b.record(stream)
+                    evs.append((a, b))
+                flush.fill_(i & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
             for layer in range(L):
                 dq[layer].copy_(hq[i][layer], non_blocking=True)
                 if appends:
@@ -455,14 +523,19 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
                     h_.copy_(d_, non_blocking=True)
             stream.synchronize()  # the step's results are on the host
         b.record(stream)
+        evs.append((a, b))
         torch.cuda.synchronize(device)
-        e_el = max_over_ranks(a.elapsed_time(b) * 1e-3, dist, device)
+        e_el = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) * 1e-3, dist, device)
         e2e = {"value": weak_scaling_value(n_e2e, ws, e_el), "unit": "steps/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
 
-    # the INT8/INT4 path alone (certification off): effective KV GB/s
+    # the INT8/INT4 path alone (certification off): effective KV GB/s, after its
+    # own warm-up steps (its kernels' first launches load their code)
     first = args.warmup + 2 * args.steps + n_e2e
+    for s in range(first, first + args.warmup):
+        run_step(s, th_naive)
+    first += args.warmup
     n_el, _ = timed(first, n_naive, th_naive, label="int8_int4")
     n_max = max_over_ranks(n_el, dist, device)
     _, nprof = timed(first + n_naive, n_naive, th_naive, profile=True, label="int8_int4_profiled")
@@ -505,7 +578,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     h2d_peak = h2d_probe_gbs(device)
 
     # per-phase algorithmic bytes per launch, from the decisions of the census
-    staged = phase_n["prefetch"] / max(1, phase_n["promote"])
+    staged = phase_n["promote_staged"] / max(1, phase_n["promote"])
     pb = phase_bytes(census, w, staged_frac=min(1.0, staged))
     phases = {}
     for p_, ms in phase_ms.items():
@@ -624,8 +697,10 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {}),
             "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
             "meta_fp16": bool(args.meta_fp16),
-            "l2": "inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (
-                t1_bytes / 2 ** 30),
+            "l2": ("inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (t1_bytes / 2 ** 30)
+                   if flush is None else
+                   "L2 flushed before each timed step (Tier 1 %.1f MiB per replica, below twice "
+                   "the %.0f MiB L2)" % (t1_bytes / 2 ** 20, l2_bytes / 2 ** 20)),
             "thresholds": dataclasses.asdict(th),
         },
         "roofline": roofline,
@@ -653,12 +728,15 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
             "rank_fail_heads": census["rank_fail"],
             "key_fail_heads": census["key_fail"],
             "heads": census["heads"],
+            "census_decodes": census["decodes"],
+            "threshold_ties": census["ties"],
             "e_key_percentiles": census["e_key_pct"],
             "e_val_percentiles": census["e_val_pct"],
         },
         "accuracy": accuracy,
         "phases": phases,
-        "gpu_launches": int(sum(v for k, v in phase_n.items() if k != "prefetch")),
+        "gpu_launches": int(sum(v for k, v in phase_n.items()
+                                if k not in ("prefetch", "promote_staged"))),
         "clocks": clk,
     }
     if e2e:
@@ -720,7 +798,7 @@ def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int 
     cache.profile_begin(1 << 20)
     run(first + naive_steps, naive_steps, th_naive)
     nms, nn, _ = cache.profile_end()
-    census = decision_census(cache, qs[warmup + cert_steps - 1], th, w, device)
+    census = decision_census(cache, [qs[warmup + cert_steps - 1]], th, w, device)
     blk_units = sum(n // BLOCK for layer in range(L) for n in cache.row_lengths(layer))
     t1_bytes = blk_units * Hkv * tier1_bytes_per_block(d, meta_fp16)
     peaks = measured_peaks()
@@ -751,7 +829,7 @@ def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int 
             "value_promoted_frac": census["value_promoted"] / max(1, census["blocks"]),
             "dense_unit_frac": census["dense_units"] / max(1, census["units"]),
             "rung_histogram": census["rungs"], "rank_fail_heads": census["rank_fail"],
-            "heads": census["heads"],
+            "heads": census["heads"], "threshold_ties": census["ties"],
             "e_key_percentiles": census["e_key_pct"], "e_val_percentiles": census["e_val_pct"],
         },
         "clocks": clk,
@@ -869,8 +947,9 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64,
-                    help="timed steps (64: the 32K workload's append-and-decode steps)")
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 64, the 32K workload's append-and-decode "
+                         "steps; 2048 for a single-layer workload, whose steps are short)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -899,6 +978,8 @@ def main(argv=None):
     ws, rank, local = dist_env()
 
     if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 64
         res = run_reference(args, w, ws, rank)
         if res is not None:
             print(json.dumps(res), flush=True)
@@ -912,6 +993,8 @@ def main(argv=None):
         barrier(dist, torch.device("cuda", local))
         build()  # no-op once rank 0 built it
     device = torch.device("cuda", local)
+    if args.steps is None:
+        args.steps = 64 if w.n_layers > 1 else 2048
     res = run_ours(args, w, ws, rank, dist, device)
     if (res is not None and ws == 1 and args.layers is None and not args.no_extra_workloads
             and w.name == DEFAULT_WORKLOAD):

@@ -263,8 +263,10 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     bulk_g2s(dst + LY::KB + LY::SB + LY::VB,
              MH ? (const void*)(t.vmeta_h + mo) : (const void*)(t.vmeta + mo), LY::MB, bar);
   };
-  if (tid == 0)
-    for (int k = 0; k < NST; ++k) issue(k);
+  // Only the first stage now: the grid's first blocks (one per CTA) then reach
+  // HBM ahead of any CTA's later stages, which thread 0 issues once block 0 has
+  // landed, so every CTA starts computing sooner.
+  if (tid == 0) issue(0);
 
   // lane roles
   const int cc = lane % CPT, tr = lane / CPT;  // logit step: channel slice, row
@@ -322,6 +324,8 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
       ok = false;
       break;
     }
+    if (tid == 0 && k == 0)
+      for (int k2 = 1; k2 < NST; ++k2) issue(k2);
     if (tid == 0 && k >= 1) {
       fence_proxy_async_smem();
       issue(k - 1 + NST);  // the previous block's stage is free
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(NT, G >= 8 ? 2 : 4)
     // let the copies still in flight land before the CTA exits, and leave empty
     // partials (the status word already reports that the results are invalid)
     if (tid == 0) {
-      const int hi = min(nblk - 1, k == 0 ? NST - 1 : k + NST - 2);
+      const int hi = min(nblk - 1, k == 0 ? 0 : k + NST - 2);
       for (int k2 = k; k2 <= hi; ++k2)
         mbar_wait(&S.bar[k2 % NST], (uint32_t)((k2 / NST) & 1), nullptr);
     }
