@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(THREADS) attend_kernel(Tier1 t, Strides st, in
         const float lb = sb * c;
         S.l[h] = S.l[h] * alpha + lb;
         float ea = S.e[h] * alpha;
-        const bool int4_here = MODE == 0 && !vprom && !sc.dense[hrow0 + h];
+        const bool int4_here = MODE == 0 && !vprom && !dh[h];  // dh[h]: head h is dense
         if (int4_here) ea += eta_b * lb;
         S.e[h] = ea;
         S.m[h] = mnew;

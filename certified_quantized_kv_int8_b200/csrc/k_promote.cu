@@ -81,10 +81,23 @@ __global__ void __launch_bounds__(THREADS) promote_kernel(Tier1 t, Strides st, i
     }
     return j1;
   };
+  const int row = tid / LPR, cl = tid - row * LPR;
+  // keys of block j: the staged device copy when it holds the block, else Tier 2
+  const __half* kunit = t.k2 + u * st.tier2;
+  const __half* sunit = kstage ? kstage + (size_t)unit * st.tier2 : nullptr;
+  auto kblock = [&](int jb) { return (jb < stage_nb ? sunit : kunit) + (size_t)jb * BLK * D; };
+  uint4 cur[NPASS], nxt[NPASS];
+  // Certified mode promotes nearly every block, so the first block's keys are
+  // requested before its flag is known (the flag and the keys then arrive
+  // together); they are reloaded in the rare case that block is not promoted.
+  if (MODE == 0) {
+    const __half* kb = kblock(j0);
+#pragma unroll
+    for (int p = 0; p < NPASS; ++p)
+      cur[p] = *reinterpret_cast<const uint4*>(kb + (size_t)(p * RPC + row) * D + cl * 8);
+  }
   int j = next_block(j0);
   if (j >= j1) return;
-
-  const int row = tid / LPR, cl = tid - row * LPR;
   float2 qr[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -97,12 +110,7 @@ __global__ void __launch_bounds__(THREADS) promote_kernel(Tier1 t, Strides st, i
     }
   }
 
-  // keys of block j: the staged device copy when it holds the block, else Tier 2
-  const __half* kunit = t.k2 + u * st.tier2;
-  const __half* sunit = kstage ? kstage + (size_t)unit * st.tier2 : nullptr;
-  auto kblock = [&](int jb) { return (jb < stage_nb ? sunit : kunit) + (size_t)jb * BLK * D; };
-  uint4 cur[NPASS], nxt[NPASS];
-  {
+  if (MODE != 0 || j != j0) {
     const __half* kb = kblock(j);
 #pragma unroll
     for (int p = 0; p < NPASS; ++p)
