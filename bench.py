@@ -202,6 +202,38 @@ def traffic_record(kernel: str):
 TIE_REL = 1e-6  # relative band of a threshold tie
 
 
+def l2_policy(w: sk.Workload, meta_fp16: bool, l2_bytes: int) -> tuple[bool, str]:
+    """Whether the timed steps flush the L2 between them (a step's Tier 1, at the
+    workload's starting lengths, below twice the L2) and the config's words for it."""
+    step_t1 = (sum(n // BLOCK for n in sk.row_lengths(w)) * w.n_layers * w.n_kv_heads
+               * tier1_bytes_per_block(w.head_dim, meta_fp16))
+    if step_t1 < 2 * l2_bytes:
+        return True, ("L2 flushed before each timed step (Tier 1 %.1f MiB per replica, below "
+                      "twice the %.0f MiB L2)" % (step_t1 / 2 ** 20, l2_bytes / 2 ** 20))
+    return False, "inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (step_t1 / 2 ** 30)
+
+
+def run_config(w: sk.Workload, ws: int, meta_fp16: bool, l2_words: str, th) -> dict:
+    """The JSON line's config, the same for both arms."""
+    appends = w.appends > 0
+    return {
+        "workload": w.name, "layers": w.n_layers, "global_batch": w.batch * ws,
+        "batch_per_gpu": w.batch, "ctx": w.ctx, "q_heads": w.n_q_heads,
+        "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+        **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {}),
+        "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
+        "meta_fp16": bool(meta_fp16), "l2": l2_words,
+        "thresholds": dataclasses.asdict(th),
+    }
+
+
+def l2_size_bytes(device=None) -> int:
+    """The GPU's L2 size (126 MiB on a B200 when no GPU is visible)."""
+    if torch.cuda.is_available():
+        return torch.cuda.get_device_properties(device or 0).L2_cache_size
+    return 126 << 20
+
+
 def decision_census(cache, qs_steps, th, w, device) -> dict:
     """Decode every layer once more with a trace, for the queries of each step in
     qs_steps (a list of per-layer query lists), and count the decisions; counts are
@@ -380,11 +412,9 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
     outs = cache.alloc_outputs()
     stream = torch.cuda.current_stream(device)
     # Tier 1 of a whole step below twice the L2: flush the L2 between steps
-    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
-    step_t1 = sum(n // BLOCK for layer in range(L) for n in lens0) * Hkv * \
-        tier1_bytes_per_block(d, args.meta_fp16)
-    flush = (torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device)
-             if step_t1 < 2 * l2_bytes else None)
+    l2_bytes = l2_size_bytes(device)
+    do_flush, l2_words = l2_policy(w, args.meta_fp16, l2_bytes)
+    flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=device) if do_flush else None
 
     # the timed loops call the C entry points with marshalled arguments prepared
     # once, so the host enqueues a layer in a few microseconds (the e2e pass below
@@ -691,18 +721,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "layers": L, "global_batch": B * ws, "batch_per_gpu": B,
-            "ctx": w.ctx, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
-            **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {}),
-            "appends_per_step": 1 if appends else 0, "parallelism": f"replicas{ws}",
-            "meta_fp16": bool(args.meta_fp16),
-            "l2": ("inputs larger than L2 (Tier 1 %.2f GiB per replica)" % (t1_bytes / 2 ** 30)
-                   if flush is None else
-                   "L2 flushed before each timed step (Tier 1 %.1f MiB per replica, below twice "
-                   "the %.0f MiB L2)" % (t1_bytes / 2 ** 20, l2_bytes / 2 ** 20)),
-            "thresholds": dataclasses.asdict(th),
-        },
+        "config": run_config(w, ws, args.meta_fp16, l2_words, th),
         "roofline": roofline,
         "roofline_kernel": roofline_kernel,
         "roofline_hbm": roofline_hbm,
@@ -933,10 +952,8 @@ def run_reference(args, w: sk.Workload, ws: int, rank: int) -> dict | None:
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per * scale * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "layers": w.n_layers, "global_batch": w.batch,
-                   "ctx": w.ctx, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim,
-                   **({"row_ctx": list(w.row_ctx)} if w.row_ctx else {})},
+        "config": run_config(w, ws, args.meta_fp16, l2_policy(w, args.meta_fp16, l2_size_bytes())[1],
+                             th),
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,

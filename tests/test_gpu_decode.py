@@ -165,9 +165,9 @@ def test_bounds_certify_the_device_output(cqa):
 
 
 @pytest.mark.parametrize("name,layers,ctx_extra", [
-    ("llama8b_32k_32layer_append", (0, 31), 0),
+    ("llama8b_32k_32layer_append", (0, 11, 31), 0),
     ("llama8b_64k_b4_t3values", (5,), 0),
-    ("llama8b_128k_needle", (17, 3), 0),
+    ("llama8b_128k_needle", (17, 3, 30), 0),
 ])
 def test_decode_full_size_sampled(cqa, name, layers, ctx_extra):
     """Full-context decode in the launch configuration of the benchmark, checked
