@@ -109,11 +109,16 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// attend grid target: four CTAs per SM
-int target_ctas(int sms) { return sms * 4; }
+// Grid target of the attention and promotion passes.  Their registers allow two
+// CTAs of 256 threads per SM.  Up to 8192 blocks of work (units x blocks) the
+// passes are latency-bound and one wave of two CTAs per SM is fastest (32K
+// context, one layer: 142 -> 136 us); above it, where the host-link reads of
+// dense heads and unstaged keys want many loads in flight, four per SM (two
+// waves) are (64K x B4: 1394 -> 1465 us with two).
+int target_ctas(int sms, long long work) { return sms * (work <= 8192 ? 2 : 4); }
 
 void chunking(int units, int nb, int sms, int* chunk_blocks, int* nchunks) {
-  int per_unit = (target_ctas(sms) + units - 1) / units;
+  int per_unit = (target_ctas(sms, (long long)units * nb) + units - 1) / units;
   if (per_unit < 1) per_unit = 1;
   int cb = nb > 0 ? (nb + per_unit - 1) / per_unit : 1;
   if (cb < 1) cb = 1;
@@ -122,10 +127,11 @@ void chunking(int units, int nb, int sms, int* chunk_blocks, int* nchunks) {
   *nchunks = nc < 1 ? 1 : nc;
 }
 
-// Partial slots per unit: the CTAs one unit may receive (a whole grid's worth
-// split over one row's kv heads, when the other rows of a ragged batch are
-// short) plus the residual block's slot.
-int max_chunks_for(int Hkv, int sms) { return target_ctas(sms) / Hkv + 2; }
+// Partial slots per unit: the most CTAs one unit may receive from the widest
+// grid, the streaming pass's four per SM (a whole grid's worth split over one
+// row's kv heads, when the other rows of a ragged batch are short), plus the
+// residual block's slot.
+int max_chunks_for(int Hkv, int sms) { return sms * 4 / Hkv + 2; }
 
 const int32_t* row_lens(const cqa_cache* c, int layer) {
   return c->len + (size_t)layer * c->cfg.batch;
