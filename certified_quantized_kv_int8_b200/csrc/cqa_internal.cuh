@@ -91,7 +91,8 @@ struct Scratch {
   int32_t* promo;    // [n_layers * B * Hkv] promoted block count per unit (pinned host, mapped)
   int* err;          // device error word (bit 0: a bounded wait gave up)
   float* part_x;     // [B*Hkv][max_chunks][G][3]  naive pass: (max Delta, residual m, residual l)
-  int* dcnt;         // [B][2] rank check: rung-3 heads, heads done (0 between calls)
+  int* dcnt;         // [B][2] rank check: rung-3 heads, heads done (0 between calls;
+                     // 8-byte aligned: one 64-bit word per row)
   size_t ls;         // logits row stride = nbm * 64 + 64
   int max_chunks;
 };

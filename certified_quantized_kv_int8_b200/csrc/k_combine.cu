@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_th
   const float* e8 = sc.ell8 + row * sh.nbm;
   const float* e16 = sc.ell16 + row * sh.nbm;
   static_assert(E >= 1 && E <= 8, "rows of at most 256 blocks");
+  const uint8_t hf0 = lane == 0 ? sc.hflags[row] : (uint8_t)0;  // loaded with the keys
   float k8[E], k16[E];
   bool pr[E];
   int np = 0;
@@ -122,10 +123,25 @@ __global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_th
   for (int k = lane; k < r; k += 32) uni[w][k] = top8[w][k];
   const int nu = base;
   __syncwarp();
-  for (int k = lane; k < nu; k += 32) {
-    const int a = uni[w][k];
-    u8[w][k] = e8[a];
-    u16[w][k] = e16[a];
+  // the union's keys from the lanes that hold them (block a: lane a % 32, slot a / 32)
+  for (int k0 = 0; k0 < nu; k0 += 32) {
+    const int k = k0 + lane;
+    const int a = k < nu ? uni[w][k] : 0;
+    const int sl = a >> 5, src = a & 31;
+    float v8 = 0.f, v16 = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float x8 = __shfl_sync(0xffffffffu, k8[i], src);
+      const float x16 = __shfl_sync(0xffffffffu, k16[i], src);
+      if (sl == i) {
+        v8 = x8;
+        v16 = x16;
+      }
+    }
+    if (k < nu) {
+      u8[w][k] = v8;
+      u16[w][k] = v16;
+    }
   }
   __syncwarp();
   // discordant pairs of U: the two orders place the pair the other way round
@@ -142,21 +158,23 @@ __global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_th
   for (int m = 16; m >= 1; m >>= 1) disc += __shfl_xor_sync(0xffffffffu, disc, m);
   const bool fail = disc > th.rank_tol;
   const bool naive = th.naive != 0;
-  int last = 0;
+  // one 64-bit arrival per head: the low word counts the row's rung-3 heads,
+  // the high word the heads done, so the last head learns both at once
+  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(sc.dcnt + 2 * b);
+  int last = 0, n3 = 0;
   if (lane == 0) {
-    uint8_t hf = sc.hflags[row];
+    uint8_t hf = hf0;
     if (!naive && fail) hf |= HF_RANKFAIL;
     sc.hflags[row] = hf;
     const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
-    if (is3) atomicAdd(&sc.dcnt[2 * b], 1);
-    __threadfence();
-    last = atomicAdd(&sc.dcnt[2 * b + 1], 1) == sh.Hq - 1;
+    __threadfence();  // this head's flags are visible before its arrival
+    const unsigned long long old = atomicAdd(cnt, (1ull << 32) + (is3 ? 1ull : 0ull));
+    last = (int)(old >> 32) == sh.Hq - 1;
+    n3 = (int)(old & 0xffffffffull) + (is3 ? 1 : 0);
   }
   if (!__shfl_sync(0xffffffffu, last, 0)) return;
   // the last head of the batch row: rung 3 per head, or rung 4 for the layer
   __threadfence();
-  int n3 = 0;
-  if (lane == 0) n3 = atomicAdd(&sc.dcnt[2 * b], 0);
   n3 = __shfl_sync(0xffffffffu, n3, 0);
   const bool layer = !naive && n3 >= need_dense;
   for (int hh = lane; hh < sh.Hq; hh += 32) {
@@ -165,10 +183,7 @@ __global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_th
     const bool is3 = !naive && (hf & (HF_KEYFAIL | HF_RANKFAIL));
     sc.dense[rw] = layer ? 4 : (is3 ? 3 : 0);
   }
-  if (lane == 0) {
-    sc.dcnt[2 * b] = 0;
-    sc.dcnt[2 * b + 1] = 0;
-  }
+  if (lane == 0) *cnt = 0ull;
 }
 
 // The same decision for rows of more than 256 blocks: one CTA of DT threads per

@@ -431,6 +431,16 @@ __global__ void __launch_bounds__(32 * G) select_small_kernel(Tier1 t, Strides s
   if (tid < G) hf_s[tid] = 0;
   if (tid == 0) npro_s = 0;
 
+  // eta_b of the blocks this thread checks for value promotion, loaded with the keys
+  constexpr int NE = (NP + NT - 1) / NT;
+  const float* eta = t.eta + u * st.eta;
+  float etv[NE];
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int j = tid + i * NT;
+    etv[i] = (!naive && j < nb) ? eta[j] : 0.f;
+  }
+
   // ---- per head: log-sum-exp, masses, Delta max; lane holds blocks lane + 32 i ----
   const float eres = sc.ell_res[hrow0 + h];
   float ev[E], dv[E], ms[E];
@@ -545,10 +555,12 @@ __global__ void __launch_bounds__(32 * G) select_small_kernel(Tier1 t, Strides s
   }
 
   // ---- rung 2: value promotion ----
-  const float* eta = t.eta + u * st.eta;
   if (!naive) {
-    for (int j = tid; j < nb; j += NT) {
-      const float e = eta[j];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const int j = tid + i * NT;
+      if (j >= nb) continue;
+      const float e = etv[i];
       uint8_t vp = 0;
       for (int hh = 0; hh < G; ++hh) {
         if (mass_all[hh][j] * e > th.v_tol) {
