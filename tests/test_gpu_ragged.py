@@ -37,20 +37,20 @@ def _fill_ragged(cache, w, layer, lens, chunk=None):
     torch.cuda.synchronize()
 
 
-def _oracle_row(w, layer, b, n):
+def _oracle_row(w, layer, b, n, fp16_meta=False):
     from oracle import build_unit
     K, V = sk.kv_row(w, layer, b, 0, n, "cpu")
-    return [build_unit(K[g].numpy(), V[g].numpy()) for g in range(w.n_kv_heads)]
+    return [build_unit(K[g].numpy(), V[g].numpy(), fp16_meta) for g in range(w.n_kv_heads)]
 
 
-def _check_decode(cache, w, layer, lens, th, step=0, label=""):
+def _check_decode(cache, w, layer, lens, th, step=0, label="", fp16_meta=False):
     from oracle import decode
     log = TieLog()
     q = sk.queries(w, layer, step, "cuda")
     res = run_decode(cache, 0, q, th)
     qc = q.cpu().numpy()
     for b, n in enumerate(lens):
-        ora = decode(qc[b], _oracle_row(w, layer, b, n), oracle_thresholds(th))
+        ora = decode(qc[b], _oracle_row(w, layer, b, n, fp16_meta), oracle_thresholds(th))
         compare_decode(row(res, b, n // 64), ora, oracle_thresholds(th), w.group, log,
                        label=f"{label} b {b} len {n}")
     for e in log.entries:
@@ -109,6 +109,30 @@ def test_ragged_decode_tiny(cqa, case):
     with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, 2048) as cache:
         _fill_ragged(cache, w, 0, TINY_LENS)
         log = _check_decode(cache, w, 0, TINY_LENS, th, label=case)
+        assert len(log.entries) <= 2
+
+
+@pytest.mark.parametrize("naive", [False, True])
+def test_ragged_fp16_meta(cqa, naive):
+    """Binary16 Tier-1 metadata with rows of different lengths appended in pieces:
+    each row's codes, scales, offsets and eta_b bit for bit against the oracle's
+    binary16 encoding of that row's tokens, then decode parity per row."""
+    from oracle import pack_int4
+    w = _tiny_batch(len(TINY_LENS))
+    th = cqa.Thresholds(**{**sk.default_thresholds(w), "tau_cov": 0.8, "naive": naive})
+    with cqa.Cache(1, w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, 2048,
+                   meta_fp16=True) as cache:
+        _fill_ragged(cache, w, 0, TINY_LENS, chunk=100)
+        arrays = {what: cache.export(0, what) for what in range(5)}
+        for b, n in enumerate(TINY_LENS):
+            for g, u in enumerate(_oracle_row(w, 0, b, n, fp16_meta=True)):
+                np.testing.assert_array_equal(arrays[0][b][g], u["kcodes"])
+                np.testing.assert_array_equal(arrays[1][b][g], u["kscale"])
+                np.testing.assert_array_equal(arrays[2][b][g], pack_int4(u["vcodes"]))
+                np.testing.assert_array_equal(arrays[3][b][g][..., 0], u["vscale"])
+                np.testing.assert_array_equal(arrays[3][b][g][..., 1], u["voffset"])
+                np.testing.assert_array_equal(arrays[4][b][g], u["eta"])
+        log = _check_decode(cache, w, 0, TINY_LENS, th, label="fp16 meta", fp16_meta=True)
         assert len(log.entries) <= 2
 
 
