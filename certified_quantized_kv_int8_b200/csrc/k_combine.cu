@@ -78,11 +78,11 @@ __global__ void __launch_bounds__(32 * DWH) decide_kernel(DecodeShape sh, cqa_th
   bool pr[E];
   int np = 0;
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
+  for (int i = 0; i < E; ++i) {  // the keys' loads do not wait for the flags'
     const int j = lane + 32 * i;
     pr[i] = j < nb && (bf[j] & BF_KEY);
-    k8[i] = pr[i] ? e8[j] : 0.f;
-    k16[i] = pr[i] ? e16[j] : 0.f;
+    k8[i] = j < nb ? e8[j] : 0.f;
+    k16[i] = j < nb ? e16[j] : 0.f;
     np += pr[i] ? 1 : 0;
   }
 #pragma unroll
