@@ -771,7 +771,7 @@ def run_ours(args, w: sk.Workload, ws: int, rank: int, dist, device) -> dict | N
 EXTRA_WORKLOADS = ("llama8b_64k_b4_t3values", "llama8b_128k_needle")
 
 
-def run_extra_workload(name: str, device, cert_steps: int = 3, naive_steps: int = 10,
+def run_extra_workload(name: str, device, cert_steps: int = 5, naive_steps: int = 10,
                        warmup: int = 3, meta_fp16: bool = False) -> dict:
     """A few timed steps of a larger workload on one GPU: certified steps/s, the
     INT8/INT4 path's effective KV GB/s and the streaming kernel's per-launch
