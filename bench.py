@@ -234,6 +234,38 @@ def l2_size_bytes(device=None) -> int:
     return 126 << 20
 
 
+def tie_counts(e_key, ell8, ell_res, rung, eta_rows, nb_row, th, G) -> dict:
+    """Decisions of one decode that sat within TIE_REL (relative) of their
+    threshold, where float32 rounding could have taken either side: heads whose
+    INT8 coverage sum at some rank (residual mass plus the largest block masses)
+    or whose E_key lies that close to tau_cov or eps_key, and (kv head, block)
+    pairs whose estimated value contribution m_b * eta_b does so for some head
+    of the group against v_tol.  e_key, rung: [B][Hq]; ell8: [B][Hq][>= nb];
+    ell_res: [B][Hq]; eta_rows[b]: [Hkv][>= nb_b]; nb_row[b]: sealed blocks."""
+    out = dict(coverage=0, e_key=0, value_promotion=0)
+    cert = rung < 3  # dense heads report 0 for both bounds
+    out["e_key"] = int((cert & (np.abs(e_key - th.eps_key) <= TIE_REL * abs(th.eps_key))).sum())
+    for b in range(len(nb_row)):
+        n = int(nb_row[b])
+        if n == 0:
+            continue
+        x = ell8[b, :, :n].astype(np.float64)  # [Hq][n]
+        er = ell_res[b].astype(np.float64)
+        mx = np.maximum(x.max(axis=1), er)
+        with np.errstate(invalid="ignore"):
+            res = np.where(np.isfinite(er), np.exp(er - mx), 0.0)
+        tot = np.exp(x - mx[:, None]).sum(axis=1) + res
+        m8 = np.exp(x - mx[:, None]) / tot[:, None]
+        cum = (res / tot)[:, None] + np.cumsum(-np.sort(-m8, axis=1), axis=1)
+        near = np.abs(cum - th.tau_cov) <= TIE_REL * th.tau_cov
+        out["coverage"] += int((near.any(axis=1) & cert[b]).sum())
+        eb = np.asarray(eta_rows[b])[:, :n]  # [Hkv][n]
+        contrib = m8.reshape(eb.shape[0], G, n) * eb[:, None, :]
+        out["value_promotion"] += int(
+            (np.abs(contrib - th.v_tol) <= TIE_REL * th.v_tol).any(axis=1).sum())
+    return out
+
+
 def decision_census(cache, qs_steps, th, w, device) -> dict:
     """Decode every layer once more with a trace, for the queries of each step in
     qs_steps (a list of per-layer query lists), and count the decisions; counts are
@@ -279,32 +311,11 @@ def decision_census(cache, qs_steps, th, w, device) -> dict:
         cert = rg < 3  # dense heads report 0 for both bounds
         e_key.append(o[1].cpu().numpy()[cert])
         e_val.append(o[2].cpu().numpy()[cert])
-        # decisions that sat within TIE_REL of their threshold (float32 rounding
-        # could have taken either side): the coverage sum at some rank, E_key, and
-        # a block's estimated value contribution
-        ek_all = o[1].cpu().numpy()
-        c["ties"]["e_key"] += int((cert & (np.abs(ek_all - th.eps_key)
-                                           <= TIE_REL * abs(th.eps_key))).sum())
-        e8 = tr["ell8"].cpu().numpy()
-        eres = tr["ell_res"].cpu().numpy()
         eta = cache.export(layer, 4)  # EXPORT_ETA: [B][Hkv][nb], or per-row arrays
-        for b in range(B):
-            n = int(nb_row[b])
-            if n == 0:
-                continue
-            x = e8[b, :, :n].astype(np.float64)  # [Hq][n]
-            mx = np.maximum(x.max(axis=1), eres[b])
-            tot = np.exp(x - mx[:, None]).sum(axis=1) + np.where(
-                np.isfinite(eres[b]), np.exp(eres[b] - mx), 0.0)
-            m8 = np.exp(x - mx[:, None]) / tot[:, None]
-            mres = np.where(np.isfinite(eres[b]), np.exp(eres[b] - mx), 0.0) / tot
-            cum = mres[:, None] + np.cumsum(-np.sort(-m8, axis=1), axis=1)
-            near = np.abs(cum - th.tau_cov) <= TIE_REL * th.tau_cov
-            c["ties"]["coverage"] += int((near.any(axis=1) & (rg[b] < 3)).sum())
-            eb = np.asarray(eta[b] if isinstance(eta, list) else eta[b])[:, :n]  # [Hkv][n]
-            contrib = m8.reshape(Hkv, G, n) * eb[:, None, :]
-            c["ties"]["value_promotion"] += int(
-                (np.abs(contrib - th.v_tol) <= TIE_REL * th.v_tol).any(axis=1).sum())
+        t = tie_counts(o[1].cpu().numpy(), tr["ell8"].cpu().numpy(), tr["ell_res"].cpu().numpy(),
+                       rg, [np.asarray(eta[b]) for b in range(B)], nb_row, th, G)
+        for k in c["ties"]:
+            c["ties"][k] += t[k]
     ek, ev = np.concatenate(e_key), np.concatenate(e_val)
     pct = (50, 90, 99, 100)
     c["e_key_pct"] = {f"p{q}": float(np.percentile(ek, q)) for q in pct} if ek.size else None

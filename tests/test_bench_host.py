@@ -96,3 +96,43 @@ def test_reference_arm_on_a_ragged_batch(capsys):
     assert rc == 0
     d = json.loads([l for l in capsys.readouterr().out.splitlines() if l.strip()][0])
     assert d["config"]["row_ctx"] == [1024, 300] and d["value"] > 0
+
+
+def test_l2_policy_and_one_config_for_both_arms(capsys):
+    """A step whose Tier 1 is below twice the L2 is timed with the L2 flushed
+    between steps; the reference arm reports the config our arm builds."""
+    import synthetic_kv as sk
+    import certified_quantized_kv_int8_b200 as cqa
+    l2 = 126 << 20
+    flush8, words8 = bench.l2_policy(sk.WORKLOADS["llama8b_8k_1layer"], False, l2)
+    flush32, words32 = bench.l2_policy(sk.WORKLOADS["llama8b_32k_32layer_append"], False, l2)
+    assert flush8 and "flushed" in words8
+    assert not flush32 and "larger than L2" in words32
+    w = sk.WORKLOADS["tiny"]
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"])
+    assert rc == 0
+    line = [l for l in capsys.readouterr().out.splitlines() if l.strip()][-1]
+    got = json.loads(line)["config"]
+    th = cqa.Thresholds(**sk.default_thresholds(w))
+    want = bench.run_config(w, 1, False, bench.l2_policy(w, False, bench.l2_size_bytes())[1], th)
+    assert got == json.loads(json.dumps(want))
+
+
+def test_tie_counts_hand_case():
+    """Residual mass 0.05 and block masses 0.5, 0.3, 0.15: the coverage sums are
+    0.55, 0.85, 1.0, so tau_cov = 0.85 is a tie for every certified head; E_key
+    equal to eps_key on one head; m_b * eta_b equal to v_tol on one block."""
+    import numpy as np
+    import certified_quantized_kv_int8_b200 as cqa
+    th = cqa.Thresholds(tau_cov=0.85, eps_key=5e-3, v_tol=0.05)
+    m = np.array([0.5, 0.3, 0.15])
+    ell8 = np.log(np.tile(m, (1, 2, 1)))           # [B=1][Hq=2][nb=3]
+    ell_res = np.log(np.full((1, 2), 0.05))
+    rung = np.array([[0, 3]])                      # head 1 went dense
+    e_key = np.array([[5e-3, 1e-2]])
+    eta = [np.array([[0.05 / 0.5, 0.0, 0.0]])]     # [Hkv=1][nb]
+    t = bench.tie_counts(e_key, ell8, ell_res, rung, eta, [3], th, G=2)
+    assert t == {"coverage": 1, "e_key": 1, "value_promotion": 1}
+    th2 = cqa.Thresholds(tau_cov=0.9, eps_key=1e-3, v_tol=0.2)
+    assert bench.tie_counts(e_key, ell8, ell_res, rung, eta, [3], th2, G=2) == \
+        {"coverage": 0, "e_key": 0, "value_promotion": 0}
