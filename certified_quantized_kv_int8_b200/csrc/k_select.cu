@@ -19,9 +19,12 @@
 // Heads with E_key > eps_key double K* (at most max_expand times).
 // A block's FP16 values are promoted when some head has m8_b * eta_b > v_tol.
 //
-// The CTA's 1024 threads form G groups, one per query head; the per-head
-// work (log-sum-exp, sort, scan, tail reductions) synchronises each group on
-// its own named barrier, and only the union steps use the whole CTA.
+// Two kernels.  Rows of up to 256 sealed blocks: one warp per query head holds
+// the head's blocks, sort keys and scan in registers (select_small_kernel).
+// Longer rows: the CTA's 1024 threads form G groups, one per query head; the
+// per-head work (log-sum-exp, sort, scan, tail reductions) synchronises each
+// group on its own named barrier, and only the union steps use the whole CTA
+// (select_kernel).
 #include "cqa_internal.cuh"
 
 namespace cqa {
